@@ -1,0 +1,360 @@
+/*
+ * stepq_oracle.c -- CPU oracle of the quantized gated Delta-rule decode step (STEPQuant).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
+ * this file; only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark do.  It shares no code with the CUDA path.
+ *
+ * It is deliberately plain and slow: loops in the order the method states its
+ * steps, all arithmetic in double precision, values that the method stores
+ * (codes, row and column scales, the output y) rounded to their storage types.
+ *
+ * Sources (web pages on STEPQuant, arXiv 2609.38169), cited by title + section:
+ *   [SUM]  hyper.ai paper summary "STEPQuant ..." -- sections "Method", "Key Contributions"
+ *   [EXP]  "Paper Explained: STEPQuant -- When and Where Quantization Errors Matter
+ *          in Delta-Rule Recurrent States" -- sections "The mechanism: rewriting state
+ *          with the delta rule", "The intuition: errors get carried forward"
+ *   [BLOG] ONTLE blog post on STEPQuant (blog.ontle.kr) -- paragraphs on the state pool,
+ *          lifetime-aware bit allocation, dual-axis fitting and the fused kernel
+ *
+ * Readings taken where the pages are silent (the pages lost every equation):
+ *   - step order: fade with the retention gate, then predict from the faded state,
+ *     then write the difference, then read out from the updated state, then
+ *     quantize for storage ([EXP] mechanism; [SUM] Method para 1);
+ *   - dual-axis fit without clipping: c_j = sqrt(max_i |S_ij|),
+ *     r_i = max_j (|S_ij| / c_j) / qmax, qmax = 2^(b-1) - 1 ([SUM] Method para 4,
+ *     impact weights dropped);
+ *   - symmetric uniform levels, nearest level with ties to even ([SUM] Method para 1, 4);
+ *   - storage: codes as offset binary u = Q + 2^(b-1) in a little-endian bit
+ *     stream of b-bit fields; element order is panel-major (16-column panels,
+ *     each panel row-major); a head block is [codes | r fp32[d_k] | c fp32[d_v]];
+ *     the pool is slot-major with heads in order inside a slot.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_PANEL 16
+
+/* ------------------------------------------------------------------------- */
+/* Sizes and layout                                                           */
+/* ------------------------------------------------------------------------- */
+
+int oracle_qmax(int bits) { return (1 << (bits - 1)) - 1; }
+
+long oracle_codes_bytes(int bits, int dk, int dv) { return (long)dk * dv * bits / 8; }
+
+long oracle_block_bytes(int bits, int dk, int dv)
+{
+    return oracle_codes_bytes(bits, dk, dv) + 4L * dk + 4L * dv;
+}
+
+/* Position of element (i, j) in the code stream: panel-major, row-major inside a panel. */
+static long stream_index(int i, int j, int dk)
+{
+    return (long)(j / ORACLE_PANEL) * dk * ORACLE_PANEL + (long)i * ORACLE_PANEL + (j % ORACLE_PANEL);
+}
+
+/* Write codes Q[dk*dv] (row-major, each in [-qmax, qmax]) as a bit stream; one bit at a time. */
+void oracle_pack_codes(int bits, int dk, int dv, const int32_t *Q, uint8_t *out)
+{
+    long nbytes = oracle_codes_bytes(bits, dk, dv);
+    memset(out, 0, (size_t)nbytes);
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            long n = stream_index(i, j, dk);
+            uint32_t u = (uint32_t)(Q[(long)i * dv + j] + (1 << (bits - 1)));
+            for (int b = 0; b < bits; b++) {
+                long bit = n * bits + b;
+                if ((u >> b) & 1u)
+                    out[bit / 8] |= (uint8_t)(1u << (bit % 8));
+            }
+        }
+}
+
+/* Inverse of oracle_pack_codes. */
+void oracle_unpack_codes(int bits, int dk, int dv, const uint8_t *in, int32_t *Q)
+{
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            long n = stream_index(i, j, dk);
+            uint32_t u = 0;
+            for (int b = 0; b < bits; b++) {
+                long bit = n * bits + b;
+                u |= (uint32_t)((in[bit / 8] >> (bit % 8)) & 1u) << b;
+            }
+            Q[(long)i * dv + j] = (int32_t)u - (1 << (bits - 1));
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Quantization: dual-axis fit + nearest level ([SUM] Method para 4)          */
+/* ------------------------------------------------------------------------- */
+
+/* Fit the scales of an fp32 state and quantize it.  Returns the number of codes
+ * that would have fallen outside [-qmax, qmax] (0 for a clip-free fit). */
+int oracle_quantize(int bits, int dk, int dv, const float *S32, int32_t *Q, float *r, float *c)
+{
+    const int qmax = oracle_qmax(bits);
+    int clipped = 0;
+    /* column scales: c_j = sqrt(max_i |S_ij|) */
+    for (int j = 0; j < dv; j++) {
+        double M = 0.0;
+        for (int i = 0; i < dk; i++) {
+            double a = fabs((double)S32[(long)i * dv + j]);
+            if (a > M) M = a;
+        }
+        c[j] = (float)sqrt(M);
+    }
+    /* row factors: r_i = max_j (|S_ij| / c_j) / qmax, over columns with c_j > 0 */
+    for (int i = 0; i < dk; i++) {
+        double m = 0.0;
+        for (int j = 0; j < dv; j++) {
+            if (c[j] > 0.0f) {
+                double t = fabs((double)S32[(long)i * dv + j]) / (double)c[j];
+                if (t > m) m = t;
+            }
+        }
+        r[i] = (float)(m / (double)qmax);
+    }
+    /* codes: nearest level, ties to even; rows or columns with zero scale get 0 */
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++) {
+            double scale = (double)r[i] * (double)c[j];
+            double x = scale > 0.0 ? (double)S32[(long)i * dv + j] / scale : 0.0;
+            double qv = nearbyint(x);
+            if (qv > qmax) { qv = qmax; clipped++; }
+            if (qv < -qmax) { qv = -qmax; clipped++; }
+            Q[(long)i * dv + j] = (int32_t)qv;
+        }
+    return clipped;
+}
+
+/* S_hat_ij = Q_ij * r_i * c_j (exact in double: <= 8-bit int times two fp32 values). */
+void oracle_dequantize(int dk, int dv, const int32_t *Q, const float *r, const float *c, double *S)
+{
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++)
+            S[(long)i * dv + j] = (double)Q[(long)i * dv + j] * (double)r[i] * (double)c[j];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Gated Delta-rule step ([EXP] mechanism)                                    */
+/* ------------------------------------------------------------------------- */
+
+/* One unquantized step on a double state S[dk*dv], in place:
+ *   fade      S'_ij = alpha_i * S_ij                (GDN: all alpha_i equal; KDA: one per key channel)
+ *   predict   u_j   = sum_i S'_ij k_i               (what the key currently retrieves)
+ *   write     d_j   = beta * (v_j - u_j);  S_ij = S'_ij + k_i d_j
+ *   read      y_j   = sum_i S_ij q_i                (from the updated state)
+ * y may be NULL. */
+void oracle_delta_step(int dk, int dv, double *S, const float *q, const float *k, const float *v,
+                       const float *alpha, float beta, double *y)
+{
+    double *u = (double *)calloc((size_t)dv, sizeof(double));
+    for (int i = 0; i < dk; i++)
+        for (int j = 0; j < dv; j++)
+            S[(long)i * dv + j] = (double)alpha[i] * S[(long)i * dv + j];
+    for (int j = 0; j < dv; j++) {
+        double s = 0.0;
+        for (int i = 0; i < dk; i++)
+            s += S[(long)i * dv + j] * (double)k[i];
+        u[j] = s;
+    }
+    for (int j = 0; j < dv; j++) {
+        double d = (double)beta * ((double)v[j] - u[j]);
+        for (int i = 0; i < dk; i++)
+            S[(long)i * dv + j] += (double)k[i] * d;
+    }
+    if (y)
+        for (int j = 0; j < dv; j++) {
+            double s = 0.0;
+            for (int i = 0; i < dk; i++)
+                s += S[(long)i * dv + j] * (double)q[i];
+            y[j] = s;
+        }
+    free(u);
+}
+
+/* One quantized decode step of one state ([SUM] Method para 1 and 4; [BLOG] per-step refit):
+ * dequantize -> delta step -> readout -> round the state to fp32 -> fit -> quantize.
+ * S_pre (optional, [dk*dv]) receives the updated state before quantization (double).
+ * Returns the clip count of the fit (0 expected). */
+int oracle_step_state(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
+                      const float *q, const float *k, const float *v, const float *alpha, float beta,
+                      int32_t *Q_out, float *r_out, float *c_out, float *y_out, double *S_pre)
+{
+    long ne = (long)dk * dv;
+    double *S = (double *)malloc((size_t)ne * sizeof(double));
+    double *y = (double *)malloc((size_t)dv * sizeof(double));
+    float *S32 = (float *)malloc((size_t)ne * sizeof(float));
+    oracle_dequantize(dk, dv, Q_in, r_in, c_in, S);
+    oracle_delta_step(dk, dv, S, q, k, v, alpha, beta, y);
+    for (int j = 0; j < dv; j++) y_out[j] = (float)y[j];
+    if (S_pre) memcpy(S_pre, S, (size_t)ne * sizeof(double));
+    for (long e = 0; e < ne; e++) S32[e] = (float)S[e];
+    int clipped = oracle_quantize(bits, dk, dv, S32, Q_out, r_out, c_out);
+    free(S); free(y); free(S32);
+    return clipped;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Pool-level drivers (slot-major pool of packed head blocks)                 */
+/* ------------------------------------------------------------------------- */
+
+/* Byte offset of each head block inside a slot, and the slot stride. */
+long oracle_head_offsets(int H, const int32_t *head_bits, int dk, int dv, long *offsets)
+{
+    long off = 0;
+    for (int h = 0; h < H; h++) {
+        offsets[h] = off;
+        off += oracle_block_bytes(head_bits[h], dk, dv);
+    }
+    return off;
+}
+
+/* Read one head block into codes + scales. */
+static void read_block(const uint8_t *blk, int bits, int dk, int dv, int32_t *Q, float *r, float *c)
+{
+    long cb = oracle_codes_bytes(bits, dk, dv);
+    oracle_unpack_codes(bits, dk, dv, blk, Q);
+    memcpy(r, blk + cb, 4L * dk);
+    memcpy(c, blk + cb + 4L * dk, 4L * dv);
+}
+
+static void write_block(uint8_t *blk, int bits, int dk, int dv, const int32_t *Q, const float *r, const float *c)
+{
+    long cb = oracle_codes_bytes(bits, dk, dv);
+    oracle_pack_codes(bits, dk, dv, Q, blk);
+    memcpy(blk + cb, r, 4L * dk);
+    memcpy(blk + cb + 4L * dk, c, 4L * dv);
+}
+
+/* One decode step for n requests over all H value heads of a pool.
+ *   pool      [num_slots * slot_stride] bytes, updated in place
+ *   slot_ids  [n]
+ *   q, k      [n, Hk, dk]; v [n, H, dv]; beta [n, H]
+ *   alpha     gate_mode 0 (GDN): [n, H];  gate_mode 1 (KDA): [n, H, dk]
+ *   y         [n, H, dv] (fp32 out)
+ * Value head h reads key head h / (H / Hk).  Returns the total clip count, or -1
+ * for an out-of-range slot id (that request is skipped). */
+long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int32_t *head_bits,
+                        int num_slots, uint8_t *pool, const int32_t *slot_ids, int n,
+                        const float *q, const float *k, const float *v, const float *alpha,
+                        const float *beta, float *y, int nthreads)
+{
+    long *offsets = (long *)malloc((size_t)H * sizeof(long));
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    long clipped = 0;
+    int bad = 0;
+    int group = H / Hk;
+    long items = (long)n * H;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(+ : clipped) reduction(| : bad)
+    for (long it = 0; it < items; it++) {
+        int b = (int)(it / H), h = (int)(it % H);
+        int slot = slot_ids[b];
+        if (slot < 0 || slot >= num_slots) { bad |= 1; continue; }
+        int bits = head_bits[h];
+        int g = h / group;
+        long ne = (long)dk * dv;
+        int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
+        int32_t *Q2 = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
+        float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
+        float *r2 = (float *)malloc(4L * dk), *c2 = (float *)malloc(4L * dv);
+        float *al = (float *)malloc(4L * dk);
+        uint8_t *blk = pool + (long)slot * stride + offsets[h];
+        read_block(blk, bits, dk, dv, Q, r, c);
+        for (int i = 0; i < dk; i++)
+            al[i] = gate_mode == 0 ? alpha[(long)b * H + h] : alpha[((long)b * H + h) * dk + i];
+        clipped += oracle_step_state(dk, dv, bits, Q, r, c,
+                                     q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
+                                     v + ((long)b * H + h) * dv, al, beta[(long)b * H + h],
+                                     Q2, r2, c2, y + ((long)b * H + h) * dv, NULL);
+        write_block(blk, bits, dk, dv, Q2, r2, c2);
+        free(Q); free(Q2); free(r); free(c); free(r2); free(c2); free(al);
+    }
+    free(offsets);
+    return bad ? -1 : clipped;
+}
+
+/* Quantize fp32 states S [n, H, dk, dv] into the slots slot_ids[n] of a pool. */
+long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_slots, uint8_t *pool,
+                      const int32_t *slot_ids, int n, const float *S, int nthreads)
+{
+    long *offsets = (long *)malloc((size_t)H * sizeof(long));
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    long clipped = 0;
+    int bad = 0;
+    long items = (long)n * H;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(+ : clipped) reduction(| : bad)
+    for (long it = 0; it < items; it++) {
+        int b = (int)(it / H), h = (int)(it % H);
+        int slot = slot_ids[b];
+        if (slot < 0 || slot >= num_slots) { bad |= 1; continue; }
+        long ne = (long)dk * dv;
+        int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
+        float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
+        clipped += oracle_quantize(head_bits[h], dk, dv, S + it * ne, Q, r, c);
+        write_block(pool + (long)slot * stride + offsets[h], head_bits[h], dk, dv, Q, r, c);
+        free(Q); free(r); free(c);
+    }
+    free(offsets);
+    return bad ? -1 : clipped;
+}
+
+/* Dequantize the slots slot_ids[n] of a pool into S [n, H, dk, dv] (fp32). */
+int oracle_pool_dump(int H, int dk, int dv, const int32_t *head_bits, int num_slots, const uint8_t *pool,
+                     const int32_t *slot_ids, int n, float *S, int nthreads)
+{
+    long *offsets = (long *)malloc((size_t)H * sizeof(long));
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    int bad = 0;
+    long items = (long)n * H;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
+    for (long it = 0; it < items; it++) {
+        int b = (int)(it / H), h = (int)(it % H);
+        int slot = slot_ids[b];
+        if (slot < 0 || slot >= num_slots) { bad |= 1; continue; }
+        long ne = (long)dk * dv;
+        int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
+        float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
+        double *Sd = (double *)malloc((size_t)ne * sizeof(double));
+        read_block(pool + (long)slot * stride + offsets[h], head_bits[h], dk, dv, Q, r, c);
+        oracle_dequantize(dk, dv, Q, r, c, Sd);
+        for (long e = 0; e < ne; e++) S[it * ne + e] = (float)Sd[e];
+        free(Q); free(r); free(c); free(Sd);
+    }
+    free(offsets);
+    return bad ? -1 : 0;
+}
+
+/* One unquantized ("FP32-state") step for a batch of double states S [n, H, dk, dv]
+ * (state index = request b, value head h; no pool, no slots).  When round_fp32 != 0
+ * the state is rounded to fp32 after the step (an fp32-stored state, as in a
+ * warm-up); otherwise it stays exact double (used for the error recursion). */
+void oracle_fp_decode_step(int H, int Hk, int dk, int dv, int gate_mode, int n, double *S,
+                           const float *q, const float *k, const float *v, const float *alpha,
+                           const float *beta, float *y, int round_fp32, int nthreads)
+{
+    int group = H / Hk;
+    long items = (long)n * H;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long it = 0; it < items; it++) {
+        int b = (int)(it / H), h = (int)(it % H);
+        int g = h / group;
+        long ne = (long)dk * dv;
+        double *Sb = S + it * ne;
+        float *al = (float *)malloc(4L * dk);
+        double *yd = (double *)malloc(8L * dv);
+        for (int i = 0; i < dk; i++)
+            al[i] = gate_mode == 0 ? alpha[(long)b * H + h] : alpha[((long)b * H + h) * dk + i];
+        oracle_delta_step(dk, dv, Sb, q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
+                          v + ((long)b * H + h) * dv, al, beta[(long)b * H + h], yd);
+        if (y)
+            for (int j = 0; j < dv; j++) y[it * dv + j] = (float)yd[j];
+        if (round_fp32)
+            for (long e = 0; e < ne; e++) Sb[e] = (double)(float)Sb[e];
+        free(al); free(yd);
+    }
+}
