@@ -1,0 +1,369 @@
+"""Benchmark of the fused quantized gated Delta-rule decode step on B200.
+
+A step is one decode step of the whole hot path (dequantize, fade, Delta write, readout,
+dual-axis refit, requantize, repack) for every (request, value head) of one batch.
+Workload: the high-concurrency GDN pool -- 512 requests scattered over a 1024-slot pool,
+32 value heads sharing 16 key heads, d_k = d_v = 128, 6-bit-nominal mixed widths from the
+lifetime-aware allocator, bf16 inputs, fp32 outputs.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Multi-GPU (torchrun): every rank owns its own pool and requests (the units are
+independent; no collective on the data path): weak scaling, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-state updates/s (req·head·step) and achieved HBM GB/s vs peak"
+UNIT = "updates/s"
+N_INPUT_SETS = 64          # distinct per-step input batches cycled through (1.1 GB on device)
+E2E_HOST_SETS = 8          # distinct pinned host batches for the end-to-end leg
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4096)
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="mixed6", choices=["mixed6", "uniform4"])
+    ap.add_argument("--e2e-steps", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_gated_delta_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as fh:
+            rec = json.load(fh)
+        if rec.get("source_hash") == kernel_source_hash() and rec.get("workload") == workload_name:
+            return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            import torch
+            ident = str(torch.cuda.get_device_properties(self.dev).uuid)
+            ident = ident if ident.startswith("GPU-") else "GPU-" + ident
+        except Exception:
+            ident = str(self.dev)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, "--query-gpu=" + q,
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def block_bytes(bits: int, dk: int = 128, dv: int = 128) -> int:
+    """Packed head block: codes (dk*dv*bits/8 bytes) + fp32 row and column factors."""
+    return dk * dv * bits // 8 + 4 * dk + 4 * dv
+
+
+def algorithmic_bytes_per_step(w, bits) -> float:
+    """State read once + written once per (request, head), plus the step's inputs and outputs."""
+    state = 2.0 * w.B * sum(block_bytes(int(b), w.dk, w.dv) for b in bits)
+    esz = 2 if w.in_dtype == 1 else 4
+    io = w.B * w.Hk * 2 * w.dk * esz            # q, k (shared by H / Hk value heads)
+    io += w.B * w.H * w.dv * esz                # v
+    io += w.B * w.H * (w.dk if w.gate_mode == 1 else 1) * esz   # alpha
+    io += w.B * w.H * esz                       # beta
+    io += w.B * w.H * w.dv * 4                  # y (fp32)
+    io += w.B * 4                               # slot ids
+    return state + io
+
+
+def _oracle_sample(w, bits, nreq: int):
+    from oracle import oracle as O
+    from quantized_gated_delta_b200 import workloads as W
+    sub = W.sample_requests(w, nreq)
+    pool = O.OraclePool(w.num_slots, bits, w.Hk, w.gate_mode)
+    xs = [{k: np.ascontiguousarray(v[sub]) for k, v in W.step_inputs(w, t).items()} for t in range(4)]
+    return pool, w.slot_ids[sub], xs
+
+
+def cpu_baseline(w, bits, seconds: float):
+    """The CPU oracle, as it stands, on this host's cores on a bounded sample of the workload."""
+    from oracle import oracle as O
+    pool, sl, xs = _oracle_sample(w, bits, 16)
+    pool.decode_step(sl, **xs[0])                        # first touch, thread start
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        pool.decode_step(sl, **xs[steps % len(xs)])
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": steps * len(sl) * w.H / el, "unit": UNIT, "cores": O.default_threads(), "kind": "oracle",
+            "sample": "%d requests x %d heads x %d decode steps of %s (%.1f s)" % (len(sl), w.H, steps, w.name, el)}
+
+
+def run_reference(args):
+    """Reference arm: the oracle, as it stands, timed on the host cores.  Each step is a
+    bounded sample of the workload's requests, sized so the whole run takes a few minutes."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from oracle import oracle as O
+    from quantized_gated_delta_b200 import workloads as W
+    w = W.make_workload(4, args.variant)
+    if w.head_bits is None:
+        bits, _ = O.allocate_bits_dp(list(w.half_life[0]), None, [4, 6, 8], w.avg_bits)
+    else:
+        bits = list(w.head_bits[0])
+    pool, sl, xs = _oracle_sample(w, bits, 16)
+    t0 = time.perf_counter()
+    pool.decode_step(sl, **xs[0])
+    per_req = (time.perf_counter() - t0) / len(sl)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nreq = int(max(1, min(16, budget // max(per_req, 1e-6))))
+    pool, sl, xs = _oracle_sample(w, bits, nreq)
+    for i in range(args.warmup):
+        pool.decode_step(sl, **xs[i % len(xs)])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        pool.decode_step(sl, **xs[i % len(xs)])
+    el = time.perf_counter() - t0
+    value = args.steps * len(sl) * w.H / el
+    cores = O.default_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "%d requests x %d heads per step, %d steps of %s"
+                                       % (len(sl), w.H, args.steps, w.name)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from quantized_gated_delta_b200 import stepq
+    from quantized_gated_delta_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = W.make_workload(4, args.variant)
+    w.seed = w.seed + 1000 * rank                    # each rank serves its own requests
+    bits = w.head_bits[0] if w.head_bits is not None else stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
+    bits = np.asarray(bits, dtype=np.uint8)
+    pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    slots = torch.from_numpy(w.slot_ids).cuda()
+
+    # per-step inputs, resident in HBM (bf16 bit patterns)
+    def dev_inputs(x):
+        return {k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).cuda() for k, v in x.items()}
+    nsets = min(N_INPUT_SETS, args.steps + args.warmup)
+    host_sets = [W.step_inputs(w, t) for t in range(nsets)]
+    sets = [dev_inputs(x) for x in host_sets]
+    y = torch.empty((w.B, w.H, w.dv), device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        x = sets[i % nsets]
+        pool.decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if pool.get_error() != 0:
+        raise RuntimeError("device flag set during warm-up")
+
+    # ---- device-timed leg: inputs resident in HBM, one kernel launch per step
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(args.warmup + i)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = t_start.elapsed_time(t_end)
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    err = pool.get_error()
+    if err != 0:
+        raise RuntimeError("device flag %d set during the timed region" % err)
+
+    units_per_step = w.B * w.H
+    value = units_per_step * args.steps * world / (ms_total / 1e3)
+    avg_kernel_s = (sum(kernel_ms) / len(kernel_ms)) / 1e3
+    alg_bytes = algorithmic_bytes_per_step(w, bits)
+    peak, peak_kind = peaks()
+    achieved = alg_bytes / avg_kernel_s / 1e9
+
+    # ---- end-to-end leg: host inputs in pinned memory, H2D + decode + D2H of y every step
+    host = []
+    for x in host_sets[:E2E_HOST_SETS]:
+        host.append({k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).pin_memory() for k, v in x.items()})
+    dbuf = {k: torch.empty_like(v, device="cuda") for k, v in host[0].items()}
+    y_host = torch.empty((w.B, w.H, w.dv), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values()) + slots.numel() * 4
+    d2h = y_host.numel() * 4
+    slots_host = torch.from_numpy(w.slot_ids).pin_memory()
+
+    def e2e_step(i):
+        hx = host[i % len(host)]
+        slots.copy_(slots_host, non_blocking=True)
+        for k in dbuf:
+            dbuf[k].copy_(hx[k], non_blocking=True)
+        pool.decode_step(slots, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], y, stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = units_per_step * args.e2e_steps * world / (ms_e2e / 1e3)
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(w, bits, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s"
+                       % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
+                          "".join(str(int(b)) for b in bits)),
+                       "avg_bits": float(np.mean(bits)), "parallelism": "dp%d (independent pools)" % world,
+                       "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
+                             % (w.B * sum(block_bytes(int(b)) for b in bits) / 1e6),
+                       "input_sets": nsets},
+            "achieved_gbs": achieved,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind,
+                         "traffic": recorded_traffic(w.name),
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "kernel": "decode_kernel", "avg_kernel_us": avg_kernel_s * 1e6},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line))
+    pool.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * stepq.h -- C ABI of libstepq: the decode step of a gated Delta-rule layer whose
+ * per-request d_k x d_v state is stored quantized (STEPQuant), for NVIDIA B200 (sm_100a).
+ *
+ * Sources, by page title and section (web pages on STEPQuant, arXiv 2609.38169):
+ *   [SUM]  hyper.ai paper summary, "Method" (symmetric uniform state quantization applied
+ *          after the update and the readout; lifetime-aware bit allocation; key-row-aware
+ *          dual-axis fitting; packed-state kernels on a recurrent-state pool)
+ *   [EXP]  "Paper Explained: STEPQuant -- When and Where Quantization Errors Matter in
+ *          Delta-Rule Recurrent States", "The mechanism: rewriting state with the delta rule"
+ *   [BLOG] ONTLE blog post on STEPQuant: per-request state pool with pre-allocated spare
+ *          slots; bit allocation, pivots and impact scores fixed offline, dual-axis scales
+ *          refit at every decoding step; the fused decode kernel
+ *
+ * Conventions
+ *   - Every function returns a status (stepq_status); 0 is success.
+ *   - A pool owns its device memory.  The caller owns every other buffer.  Unless stated
+ *     otherwise, tensor arguments are DEVICE pointers to contiguous row-major arrays, and
+ *     must be 16-byte aligned.
+ *   - Calls that take a stream enqueue work on it and return without synchronizing; an
+ *     asynchronous CUDA fault surfaces as STEPQ_CUDA_ERROR on a later call.  A pool must
+ *     not be used on two streams at once without synchronization by the caller.
+ *   - slot_ids within one call must be distinct; duplicates give undefined results.  An
+ *     out-of-range slot id is skipped by the kernels and raises the pool's sticky device
+ *     flag (read with stepq_pool_get_error); kernels never trap.
+ *
+ * State and layout (shared by every call; the pages leave the format open)
+ *   - value head h of request b lives in slot s = slot_ids[b]; key head g(h) = h / (H / H_k)
+ *   - the pool is slot-major; inside a slot the value heads follow in order; a head block is
+ *       codes | r[d_k] float32 | c[d_v] float32
+ *     with the head's bit width b in {4, 6, 8}; block sizes 9216, 13312, 17408 bytes for
+ *     d_k = d_v = 128 (all multiples of 128 bytes)
+ *   - a state is S_ij ~= Q_ij * r_i * c_j with integer codes |Q_ij| <= qmax = 2^(b-1) - 1
+ *   - codes are stored as offset binary u = Q + 2^(b-1) in a little-endian bit stream of
+ *     b-bit fields (4-bit: two per byte, low nibble first; 6-bit: four per three bytes;
+ *     8-bit: one per byte); the element order in the stream is panel-major: 16-column
+ *     panels, each panel row-major, i.e. stream index = (j / 16) * d_k * 16 + i * 16 + j % 16
+ *   - a zero-filled block (r = c = 0) is the zero state
+ */
+#ifndef STEPQ_H
+#define STEPQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define STEPQ_API __attribute__((visibility("default")))
+#else
+#define STEPQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                      /* same type as cudaStream_t; NULL = legacy stream */
+typedef struct CUstream_st *stepq_stream;
+
+typedef enum {
+    STEPQ_OK = 0,
+    STEPQ_INVALID_ARG = -1,              /* null pointer, bad size or alignment, bad count   */
+    STEPQ_OUT_OF_MEMORY = -2,            /* device or host allocation failed                 */
+    STEPQ_CUDA_ERROR = -3,               /* a CUDA runtime call or kernel launch failed      */
+    STEPQ_UNSUPPORTED = -4,              /* d_k or d_v != 128, or a bit width not in {4,6,8} */
+    STEPQ_DEVICE_FLAG = -5               /* the pool's sticky device flag was set            */
+} stepq_status;
+
+enum { STEPQ_GATE_GDN = 0, STEPQ_GATE_KDA = 1 };
+enum { STEPQ_DTYPE_F32 = 0, STEPQ_DTYPE_BF16 = 1 };
+
+/* Bits of the sticky device flag. */
+enum {
+    STEPQ_FLAG_BAD_SLOT = 1,             /* a slot id outside [0, num_slots) was skipped     */
+    STEPQ_FLAG_TIMEOUT = 2               /* a bounded wait inside a kernel gave up           */
+};
+
+typedef struct stepq_pool stepq_pool;
+
+typedef struct {
+    int32_t num_slots;                   /* pool slots (requests resident at once + spares)  */
+    int32_t num_heads;                   /* value heads H                                    */
+    int32_t num_key_heads;               /* key heads H_k, divides H                         */
+    int32_t d_k, d_v;                    /* state shape; 128 x 128 is supported              */
+    int32_t gate_mode;                   /* STEPQ_GATE_GDN: alpha [n, H];
+                                            STEPQ_GATE_KDA: alpha [n, H, d_k]                 */
+    int32_t in_dtype;                    /* STEPQ_DTYPE_F32 or _BF16: dtype of q, k, v,
+                                            alpha and beta (y is always float32)             */
+    const uint8_t *head_bits;            /* HOST array [H], each 4, 6 or 8 (from an offline
+                                            allocation, e.g. stepq_allocate_bits)            */
+} stepq_pool_desc;
+
+/* Create a pool and zero it (every slot holds the zero state).  The descriptor and
+ * head_bits are copied.  Synchronizes the device.  [BLOG: pool with spare slots] */
+STEPQ_API int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out);
+
+/* Free the pool and its device memory.  Synchronizes the device.  NULL is a no-op. */
+STEPQ_API int stepq_pool_destroy(stepq_pool *pool);
+
+/* Bytes of one slot and of the whole pool (host outputs; either may be NULL). */
+STEPQ_API int stepq_pool_bytes(const stepq_pool *pool, size_t *slot_stride, size_t *total);
+
+/* Byte offset of value head h's block inside a slot (host output). */
+STEPQ_API int stepq_pool_head_offset(const stepq_pool *pool, int32_t h, size_t *offset);
+
+/* Quantize fp32 states into slots: S [n, H, d_k, d_v] float32 (device).  Per state:
+ * clip-free dual-axis fit c_j = sqrt(max_i |S_ij|), r_i = max_j (|S_ij| / c_j) / qmax,
+ * then Q_ij = nearest level of S_ij / (r_i c_j), ties to even.  [SUM Method: fitting] */
+STEPQ_API int stepq_pool_load_fp32(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const float *S,
+                         stepq_stream stream);
+
+/* Copy packed slot images into slots: bytes [n, slot_stride] (device), e.g. from
+ * stepq_pool_dump_packed or a checkpoint.  Restores states bit for bit. */
+STEPQ_API int stepq_pool_load_packed(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
+                           const uint8_t *bytes, stepq_stream stream);
+
+/* Dequantize slots: S_out [n, H, d_k, d_v] float32 (device), S_ij = Q_ij * r_i * c_j. */
+STEPQ_API int stepq_pool_dump_fp32(const stepq_pool *pool, const int32_t *slot_ids, int32_t n, float *S_out,
+                         stepq_stream stream);
+
+/* Copy slot images out: bytes_out [n, slot_stride] (device). */
+STEPQ_API int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot_ids, int32_t n,
+                           uint8_t *bytes_out, stepq_stream stream);
+
+/* One decode step for n requests, every value head, in one fused kernel.
+ * Per (request b, value head h), with S the state in slot slot_ids[b]:
+ *   dequantize S_ij = Q_ij r_i c_j;  fade S'_ij = alpha_i S_ij (GDN: one alpha per head;
+ *   KDA: one per key channel);  predict u = S'^T k;  write S = S' + k (beta (v - u))^T;
+ *   read y = S^T q from the updated, unquantized state;  refit r, c;  requantize to the
+ *   head's width with round-half-even;  repack in place.       [EXP mechanism; SUM Method]
+ * Arguments (device, in_dtype unless noted):
+ *   q, k   [n, H_k, d_k]     query and key (used as given: no normalization or scaling)
+ *   v      [n, H, d_v]
+ *   alpha  [n, H] (GDN) or [n, H, d_k] (KDA): retention in (0, 1], not its logarithm
+ *   beta   [n, H]
+ *   y      [n, H, d_v] float32 output; rows of skipped (bad-slot) requests are not written
+ * n = 0 is a valid no-op. */
+STEPQ_API int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q,
+                      const void *k, const void *v, const void *alpha, const void *beta, float *y,
+                      stepq_stream stream);
+
+/* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
+ * Synchronizes the device. */
+STEPQ_API int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out);
+
+/* Lifetime-aware bit allocation (host, offline).             [SUM Method, para 2; BLOG]
+ * For each unit u (a head): retention rho_u = 2^(-1 / half_life[u]) (the mean log
+ * retention of the unit), lifetime weight w_u = 1 / (1 - rho_u) (error retention after j
+ * updates ~ rho^j, summed); distortion D_u(b) = distortion[u * C + c] for candidate
+ * cand[c], or, when distortion is NULL, 2^(-2 b) (a uniform quantizer's error power).
+ * Chooses bits_out[u] in cand minimising sum_u w_u D_u(bits_out[u]) subject to
+ * sum_u bits_out[u] <= floor(N * avg_bits), by exact dynamic programming.
+ * All pointers are HOST pointers.  half_life must be finite and > 0; cand must be
+ * distinct widths in {4, 6, 8}.  Returns STEPQ_INVALID_ARG when no assignment fits. */
+STEPQ_API int stepq_allocate_bits(const double *half_life, const double *distortion, int32_t N,
+                        const uint8_t *cand, int32_t C, double avg_bits, uint8_t *bits_out);
+
+/* Static description of a status code. */
+STEPQ_API const char *stepq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STEPQ_H */

@@ -1,0 +1,211 @@
+// stepq_capi.cu -- the C ABI of libstepq (declared in include/stepq.h): pool
+// management, argument validation and kernel launches.  Every step of the decode
+// path runs in the kernels of stepq_kernels.cu; this file only checks and launches.
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "stepq_internal.h"
+#include "stepq_tile.cuh"
+
+using stepq::block_bytes;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int status_of(cudaError_t e)
+{
+    if (e == cudaSuccess) return STEPQ_OK;
+    if (e == cudaErrorMemoryAllocation) return STEPQ_OUT_OF_MEMORY;
+    return STEPQ_CUDA_ERROR;
+}
+
+// The pool's device must be current for every call that touches it.
+int check_device(const stepq_pool *p)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return STEPQ_CUDA_ERROR;
+    return dev == p->device ? STEPQ_OK : STEPQ_INVALID_ARG;
+}
+
+int check_slots(const stepq_pool *p, const int32_t *slot_ids, int32_t n)
+{
+    if (!p || n < 0) return STEPQ_INVALID_ARG;
+    if (n > 0 && (!slot_ids || !aligned_to(slot_ids, 4))) return STEPQ_INVALID_ARG;
+    if (n > p->num_slots || n > 65535) return STEPQ_INVALID_ARG;
+    return check_device(p);
+}
+
+void free_pool(stepq_pool *p)
+{
+    if (!p) return;
+    cudaFree(p->d_pool);
+    cudaFree(p->d_offs);
+    cudaFree(p->d_bits);
+    cudaFree(p->d_flag);
+    delete p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *stepq_status_string(int status)
+{
+    switch (status) {
+    case STEPQ_OK: return "ok";
+    case STEPQ_INVALID_ARG: return "invalid argument";
+    case STEPQ_OUT_OF_MEMORY: return "out of memory";
+    case STEPQ_CUDA_ERROR: return "CUDA error";
+    case STEPQ_UNSUPPORTED: return "unsupported configuration (d_k = d_v = 128, bits in {4, 6, 8})";
+    case STEPQ_DEVICE_FLAG: return "device flag set (bad slot id or kernel wait timeout)";
+    default: return "unknown status";
+    }
+}
+
+int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
+{
+    if (!desc || !out || !desc->head_bits) return STEPQ_INVALID_ARG;
+    *out = nullptr;
+    if (desc->num_slots <= 0 || desc->num_heads <= 0 || desc->num_key_heads <= 0) return STEPQ_INVALID_ARG;
+    if (desc->num_heads % desc->num_key_heads != 0) return STEPQ_INVALID_ARG;
+    if (desc->num_heads > stepq::kMaxHeads) return STEPQ_UNSUPPORTED;
+    if (desc->gate_mode != STEPQ_GATE_GDN && desc->gate_mode != STEPQ_GATE_KDA) return STEPQ_INVALID_ARG;
+    if (desc->in_dtype != STEPQ_DTYPE_F32 && desc->in_dtype != STEPQ_DTYPE_BF16) return STEPQ_INVALID_ARG;
+    if (desc->d_k != stepq::DK || desc->d_v != stepq::DV) return STEPQ_UNSUPPORTED;
+    for (int h = 0; h < desc->num_heads; ++h) {
+        const int b = desc->head_bits[h];
+        if (b != 4 && b != 6 && b != 8) return STEPQ_UNSUPPORTED;
+    }
+    stepq_pool *p = new (std::nothrow) stepq_pool();
+    if (!p) return STEPQ_OUT_OF_MEMORY;
+    p->num_slots = desc->num_slots;
+    p->H = desc->num_heads;
+    p->Hk = desc->num_key_heads;
+    p->gate_mode = desc->gate_mode;
+    p->in_dtype = desc->in_dtype;
+    p->bits.assign(desc->head_bits, desc->head_bits + p->H);
+    p->offs.resize(p->H);
+    long long off = 0;
+    for (int h = 0; h < p->H; ++h) {
+        p->offs[h] = off;
+        off += block_bytes(p->bits[h]);
+        if (block_bytes(p->bits[h]) > p->max_block) p->max_block = block_bytes(p->bits[h]);
+    }
+    p->slot_stride = off;
+    p->total = off * (long long)p->num_slots;
+    cudaError_t e = cudaGetDevice(&p->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_pool, size_t(p->total));
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_offs, sizeof(long long) * p->H);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_bits, size_t(p->H));
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_flag, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(p->d_pool, 0, size_t(p->total));
+    if (e == cudaSuccess) e = cudaMemset(p->d_flag, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpy(p->d_offs, p->offs.data(), sizeof(long long) * p->H, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(p->d_bits, p->bits.data(), size_t(p->H), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = stepq::decode_configure(p);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        free_pool(p);
+        return status_of(e);
+    }
+    *out = p;
+    return STEPQ_OK;
+}
+
+int stepq_pool_destroy(stepq_pool *pool)
+{
+    if (!pool) return STEPQ_OK;
+    const cudaError_t e = cudaDeviceSynchronize();
+    free_pool(pool);
+    return status_of(e);
+}
+
+int stepq_pool_bytes(const stepq_pool *pool, size_t *slot_stride, size_t *total)
+{
+    if (!pool) return STEPQ_INVALID_ARG;
+    if (slot_stride) *slot_stride = size_t(pool->slot_stride);
+    if (total) *total = size_t(pool->total);
+    return STEPQ_OK;
+}
+
+int stepq_pool_head_offset(const stepq_pool *pool, int32_t h, size_t *offset)
+{
+    if (!pool || !offset || h < 0 || h >= pool->H) return STEPQ_INVALID_ARG;
+    *offset = size_t(pool->offs[h]);
+    return STEPQ_OK;
+}
+
+int stepq_pool_load_fp32(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const float *S,
+                         stepq_stream stream)
+{
+    int st = check_slots(pool, slot_ids, n);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!S || !aligned16(S)) return STEPQ_INVALID_ARG;
+    return status_of(stepq::launch_load_fp32(pool, slot_ids, n, S, stream));
+}
+
+int stepq_pool_load_packed(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const uint8_t *bytes,
+                           stepq_stream stream)
+{
+    int st = check_slots(pool, slot_ids, n);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!bytes || !aligned16(bytes)) return STEPQ_INVALID_ARG;
+    return status_of(stepq::launch_copy_slots(pool, slot_ids, n, bytes, nullptr, true, stream));
+}
+
+int stepq_pool_dump_fp32(const stepq_pool *pool, const int32_t *slot_ids, int32_t n, float *S_out,
+                         stepq_stream stream)
+{
+    int st = check_slots(pool, slot_ids, n);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!S_out || !aligned16(S_out)) return STEPQ_INVALID_ARG;
+    return status_of(stepq::launch_dump_fp32(pool, slot_ids, n, S_out, stream));
+}
+
+int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot_ids, int32_t n, uint8_t *bytes_out,
+                           stepq_stream stream)
+{
+    int st = check_slots(pool, slot_ids, n);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!bytes_out || !aligned16(bytes_out)) return STEPQ_INVALID_ARG;
+    return status_of(stepq::launch_copy_slots(pool, slot_ids, n, nullptr, bytes_out, false, stream));
+}
+
+int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q, const void *k,
+                      const void *v, const void *alpha, const void *beta, float *y, stepq_stream stream)
+{
+    int st = check_slots(pool, slot_ids, n);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!q || !k || !v || !alpha || !beta || !y) return STEPQ_INVALID_ARG;
+    // q, k, v (and the KDA gate) are bulk-copied: 16-byte aligned rows
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned_to(y, 4)) return STEPQ_INVALID_ARG;
+    const size_t esz = pool->in_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
+    if (pool->gate_mode == STEPQ_GATE_KDA ? !aligned16(alpha) : !aligned_to(alpha, esz)) return STEPQ_INVALID_ARG;
+    if (!aligned_to(beta, esz)) return STEPQ_INVALID_ARG;
+    return status_of(stepq::launch_decode(pool, slot_ids, n, q, k, v, alpha, beta, y, stream));
+}
+
+int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out)
+{
+    if (!pool || !flag_out) return STEPQ_INVALID_ARG;
+    int st = check_device(pool);
+    if (st != STEPQ_OK) return st;
+    int h = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&h, pool->d_flag, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(pool->d_flag, 0, sizeof(int));
+    if (e != cudaSuccess) return status_of(e);
+    *flag_out = h;
+    return STEPQ_OK;
+}
+
+}  // extern "C"

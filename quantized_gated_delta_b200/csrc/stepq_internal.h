@@ -1,0 +1,45 @@
+// stepq_internal.h -- pool object and kernel launchers shared by the C ABI and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <vector>
+#include <cuda_runtime.h>
+
+#include "stepq.h"
+
+struct stepq_pool {
+    int32_t num_slots = 0, H = 0, Hk = 0, gate_mode = 0, in_dtype = 0;
+    std::vector<uint8_t> bits;          // [H]
+    std::vector<long long> offs;        // [H] byte offset of each head block in a slot
+    long long slot_stride = 0;          // bytes per slot
+    long long total = 0;                // bytes of the pool
+    int max_block = 0;                  // largest head block (bytes)
+    int device = 0;
+    int num_sms = 0;
+    uint8_t *d_pool = nullptr;          // [num_slots * slot_stride]
+    long long *d_offs = nullptr;        // [H]
+    uint8_t *d_bits = nullptr;          // [H]
+    int *d_flag = nullptr;              // sticky device flag (STEPQ_FLAG_* bits)
+    int decode_grid = 0;                // persistent CTAs for the decode kernel
+    size_t decode_smem = 0;             // dynamic shared memory of the decode kernel
+    int stage_bytes = 0;
+    int blk_cap = 0;
+};
+
+namespace stepq {
+
+constexpr int kMaxHeads = 256;
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t decode_configure(stepq_pool *p);
+cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, const void *q,
+                          const void *k, const void *v, const void *alpha, const void *beta,
+                          float *y, cudaStream_t stream);
+cudaError_t launch_load_fp32(const stepq_pool *p, const int32_t *slot_ids, int n, const float *S,
+                             cudaStream_t stream);
+cudaError_t launch_dump_fp32(const stepq_pool *p, const int32_t *slot_ids, int n, float *S,
+                             cudaStream_t stream);
+cudaError_t launch_copy_slots(const stepq_pool *p, const int32_t *slot_ids, int n, const uint8_t *src,
+                              uint8_t *dst, bool into_pool, cudaStream_t stream);
+
+}  // namespace stepq

@@ -170,14 +170,15 @@ def step_inputs(w: Workload, t: int, phase: int = PHASE_RUN, layer: int = 0) -> 
     [B, H, dk] (KDA)."""
     r = _rng(w.seed, layer, phase, t)
     B, H, Hk, dk, dv = w.B, w.H, w.Hk, w.dk, w.dv
-    q = r.standard_normal((B, Hk, dk))
-    k = r.standard_normal((B, Hk, dk))
-    q /= np.linalg.norm(q, axis=-1, keepdims=True)
-    k /= np.linalg.norm(k, axis=-1, keepdims=True)
-    v = r.standard_normal((B, H, dv))
-    beta = 1.0 / (1.0 + np.exp(-r.standard_normal((B, H))))
+    f32 = np.float32
+    q = r.standard_normal((B, Hk, dk), dtype=f32)
+    k = r.standard_normal((B, Hk, dk), dtype=f32)
+    q /= np.sqrt(np.einsum("bhd,bhd->bh", q, q))[..., None]
+    k /= np.sqrt(np.einsum("bhd,bhd->bh", k, k))[..., None]
+    v = r.standard_normal((B, H, dv), dtype=f32)
+    beta = 1.0 / (1.0 + np.exp(-r.standard_normal((B, H), dtype=f32)))
     if w.gate_mode == GATE_GDN:
-        alpha = np.broadcast_to(2.0 ** (-1.0 / w.half_life[layer]), (B, H))
+        alpha = np.broadcast_to((2.0 ** (-1.0 / w.half_life[layer])).astype(f32), (B, H))
     else:
         x = r.standard_normal((B, H, dk)) + w.kda_mu[layer][None, :, None]
         alpha = np.exp(-_softplus(x))

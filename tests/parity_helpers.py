@@ -1,0 +1,90 @@
+"""Shared helpers of the GPU parity tests: workload set-up on the oracle side, moving
+inputs to the device, and comparison of packed states (codes +-1 rule, scale ulps)."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import oracle as O
+from quantized_gated_delta_b200 import workloads as W
+
+# Tolerances (the reading of the single-step bar; see the design notes):
+CODE_FLIP_RATE = 1e-5       # codes may differ by exactly 1 at this rate
+R_ULP = 8                   # row factors r within 8 ulp of the oracle's
+C_ULP = 4                   # column factors c within 4 ulp
+Y_MAX_REL = 1e-4            # per (request, head): max_j |dy_j| / max_j |y_j|
+Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
+
+
+def head_bits(w: W.Workload, layer: int = 0) -> np.ndarray:
+    """Fixed widths of the workload, else the oracle's lifetime-aware allocation."""
+    if w.head_bits is not None:
+        return np.asarray(w.head_bits[layer], dtype=np.int32)
+    bits, _ = O.allocate_bits_dp(list(w.half_life[layer]), None, [4, 6, 8], w.avg_bits)
+    return np.asarray(bits, dtype=np.int32)
+
+
+def sub_inputs(x: dict, idx) -> dict:
+    return {k: np.ascontiguousarray(v[idx]) for k, v in x.items()}
+
+
+def oracle_pool_with_warmup(w: W.Workload, bits, req_idx, layer: int = 0) -> O.OraclePool:
+    """Oracle pool whose slots slot_ids[req_idx] hold the quantized state reached after the
+    workload's FP32 warm-up steps (unquantized steps from zero, fp32-stored)."""
+    pool = O.OraclePool(w.num_slots, bits, w.Hk, w.gate_mode)
+    req_idx = np.asarray(req_idx)
+    S = np.zeros((len(req_idx), w.H, w.dk, w.dv))
+    for t in range(w.warmup_steps):
+        x = sub_inputs(W.step_inputs(w, t, W.PHASE_WARMUP, layer), req_idx)
+        O.fp_decode_step(S, w.Hk, w.gate_mode, x["q"], x["k"], x["v"], x["alpha"], x["beta"],
+                         round_fp32=True)
+    pool.load_fp32(w.slot_ids[req_idx], S.astype(np.float32))
+    return pool
+
+
+def to_device(w: W.Workload, x: dict, torch):
+    """Inputs of one step as CUDA tensors in the device dtype (bf16 as its bit patterns)."""
+    out = {}
+    for key, val in x.items():
+        a = W.as_device_dtype(w, val)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        out[key] = t.cuda()
+    return out
+
+
+def ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in units in the last place between same-signed float32 arrays."""
+    ia = a.astype(np.float32).view(np.int32).astype(np.int64)
+    ib = b.astype(np.float32).view(np.int32).astype(np.int64)
+    return np.abs(ia - ib)
+
+
+def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv=128) -> dict:
+    """Compare slot images [n, slot_stride] head by head."""
+    offs, stride = O.head_offsets(bits, dk, dv)
+    res = dict(max_code_diff=0, flips=0, elements=0, r_ulp=0, c_ulp=0, byte_equal=True)
+    for s in range(gpu_bytes.shape[0]):
+        for h, b in enumerate(bits):
+            o = int(offs[h])
+            n = O.block_bytes(int(b), dk, dv)
+            g, r = gpu_bytes[s, o:o + n], ora_bytes[s, o:o + n]
+            if np.array_equal(g, r):
+                res["elements"] += dk * dv
+                continue
+            res["byte_equal"] = False
+            Qg, rg, cg = O.split_block(g, int(b), dk, dv)
+            Qo, ro, co = O.split_block(r, int(b), dk, dv)
+            d = np.abs(Qg - Qo)
+            res["max_code_diff"] = max(res["max_code_diff"], int(d.max()))
+            res["flips"] += int((d > 0).sum())
+            res["elements"] += d.size
+            res["r_ulp"] = max(res["r_ulp"], int(ulp_diff(rg, ro).max()))
+            res["c_ulp"] = max(res["c_ulp"], int(ulp_diff(cg, co).max()))
+    return res
+
+
+def y_max_rel(yg: np.ndarray, yo: np.ndarray) -> float:
+    """Largest per-(request, head) max_j |dy_j| / max_j |y_j| (y shaped [..., dv])."""
+    num = np.abs(yg - yo).max(axis=-1)
+    den = np.abs(yo).max(axis=-1)
+    den = np.where(den > 0, den, 1.0)
+    return float((num / den).max())

@@ -1,0 +1,102 @@
+"""Host-side checks of the C ABI (no GPU work): the library builds and loads, exports
+every entry point declared in include/stepq.h, rejects bad descriptors before touching
+the device, and its bit allocator equals the oracle's."""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def S():
+    from quantized_gated_delta_b200 import build, stepq
+    build.build()
+    stepq.load_library()
+    return stepq
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"STEPQ_API\s+[\w\s\*]*?\b(stepq_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(S):
+    names = declared_symbols()
+    assert len(names) >= 12
+    lib = S.load_library()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(S.EXPORTED) <= names
+
+
+def test_status_strings(S):
+    for st in (0, -1, -2, -3, -4, -5):
+        assert S.stepq_status_string(st)
+    assert "unknown" in S.stepq_status_string(42)
+
+
+def test_descriptor_validation_before_device(S):
+    import ctypes
+    lib = S.load_library()
+    out = ctypes.c_void_p()
+    assert lib.stepq_pool_create(None, ctypes.byref(out)) == -1
+    bits = np.array([4, 6, 8, 5], np.uint8)
+    d = S.stepq_pool_desc(4, 4, 2, 128, 128, 0, 1, bits.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    assert lib.stepq_pool_create(ctypes.byref(d), ctypes.byref(out)) == -4     # width 5
+    bits[3] = 8
+    d.d_k = 64
+    assert lib.stepq_pool_create(ctypes.byref(d), ctypes.byref(out)) == -4     # d_k != 128
+    d.d_k = 128
+    d.num_key_heads = 3
+    assert lib.stepq_pool_create(ctypes.byref(d), ctypes.byref(out)) == -1     # Hk does not divide H
+    d.num_key_heads = 2
+    d.gate_mode = 7
+    assert lib.stepq_pool_create(ctypes.byref(d), ctypes.byref(out)) == -1
+    assert lib.stepq_pool_destroy(None) == 0
+    assert lib.stepq_pool_bytes(None, None, None) == -1
+    assert lib.stepq_decode_step(None, None, 0, None, None, None, None, None, None, None) == -1
+
+
+@pytest.mark.parametrize("N", [1, 3, 6, 8])
+def test_allocator_equals_exhaustive_search(S, N):
+    rng = np.random.default_rng(40 + N)
+    for trial in range(5):
+        hl = np.exp(rng.uniform(0, math.log(4096), N))
+        dist = None if trial % 2 == 0 else np.sort(rng.lognormal(0, 1, (N, 3)))[:, ::-1] * np.array([1, 0.1, 0.01])
+        avg = [5.0, 6.0, 7.0, 4.5, 6.5][trial]
+        ref, _ = O.allocate_bits_bruteforce(list(hl), dist, [4, 6, 8], avg)
+        got = S.stepq_allocate_bits(hl, dist, (4, 6, 8), avg)
+        assert list(got) == ref
+
+
+def test_allocator_equals_oracle_dp_at_layer_size(S):
+    rng = np.random.default_rng(50)
+    for _ in range(10):
+        hl = np.exp(rng.uniform(0, math.log(4096), 32))
+        ref, _ = O.allocate_bits_dp(list(hl), None, [4, 6, 8], 6.0)
+        got = S.stepq_allocate_bits(hl)
+        assert list(got) == ref and got.mean() == 6.0
+
+
+def test_allocator_candidate_order_and_errors(S):
+    hl = [2.0, 50.0, 4000.0]
+    a = S.stepq_allocate_bits(hl, None, (8, 4, 6), 6.0)
+    b = S.stepq_allocate_bits(hl, None, (4, 6, 8), 6.0)
+    assert list(a) == list(b) == [4, 6, 8]
+    with pytest.raises(S.StepqError):
+        S.stepq_allocate_bits(hl, None, (4, 6, 8), 3.0)        # budget below 4 bits per unit
+    with pytest.raises(S.StepqError):
+        S.stepq_allocate_bits([1.0, -2.0], None, (4, 8), 6.0)  # negative half-life
+    with pytest.raises(S.StepqError):
+        S.stepq_allocate_bits([1.0], None, (4, 4), 6.0)        # duplicate candidate

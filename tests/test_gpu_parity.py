@@ -1,0 +1,322 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs.  Every test here needs a B200 and the built libstepq.so."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from quantized_gated_delta_b200 import workloads as W
+from tests import parity_helpers as PH
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+f32 = np.float32
+
+
+@pytest.fixture(scope="module")
+def S():
+    from quantized_gated_delta_b200 import stepq
+    stepq.load_library()
+    return stepq
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.cuda() if dtype is None else t.to(dtype).cuda()
+
+
+def slots_t(ids):
+    return dev(np.asarray(ids, dtype=np.int32))
+
+
+def dump_bytes(pool, ids):
+    out = torch.empty((len(ids), pool.slot_stride), dtype=torch.uint8, device="cuda")
+    pool.dump_packed(slots_t(ids), out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def load_bytes(pool, ids, data):
+    pool.load_packed(slots_t(ids), dev(data))
+
+
+def unit(rng, n):
+    x = rng.standard_normal(n)
+    return (x / np.linalg.norm(x)).astype(f32)
+
+
+def random_states(rng, n, H, steps=24, alpha=0.98):
+    S_ = np.zeros((n, H, 128, 128))
+    q = np.zeros((n, H, 128), f32)
+    for _ in range(steps):
+        x = dict(q=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+                 k=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+                 v=rng.standard_normal((n, H, 128)).astype(f32),
+                 alpha=np.full((n, H), alpha, f32), beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+        O.fp_decode_step(S_, H, 0, x["q"], x["k"], x["v"], x["alpha"], x["beta"], round_fp32=True)
+    return S_.astype(f32)
+
+
+# --------------------------------------------------------------------------- pool I/O
+
+def test_load_fp32_matches_oracle_quantize(S):
+    rng = np.random.default_rng(1)
+    bits = [4, 6, 8, 8, 6, 4]
+    n = 5
+    st = random_states(rng, n, len(bits))
+    st[0, 0, 3, :] = 0                      # zero row
+    st[0, 1, :, 9] = 0                      # zero column
+    st[1, 2, 7, 11] *= -50                  # outlier
+    st[2, 3] = 0                            # all-zero state
+    st[3, 4] *= 1e-30                       # tiny magnitudes
+    st[4, 5] *= 1e20                        # huge magnitudes
+    ids = np.array([7, 2, 0, 5, 3], np.int32)
+    op = O.OraclePool(8, bits, len(bits))
+    op.load_fp32(ids, st)
+    gp = S.Pool(8, bits, len(bits), S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    gp.load_fp32(slots_t(ids), dev(st))
+    res = PH.compare_slots(dump_bytes(gp, ids), op.slot_bytes(ids), bits)
+    assert gp.get_error() == 0
+    assert res["max_code_diff"] <= 1
+    assert res["flips"] <= PH.CODE_FLIP_RATE * res["elements"] + 1e-12 or res["flips"] <= 1
+    assert res["c_ulp"] == 0               # c = sqrt(max |S|): both sides correctly rounded
+    assert res["r_ulp"] <= PH.R_ULP
+    # untouched slots stay zero
+    z = dump_bytes(gp, [1, 4, 6])
+    assert not z.any()
+
+
+def test_dump_fp32_is_exact(S):
+    rng = np.random.default_rng(2)
+    bits = [8, 4, 6]
+    st = random_states(rng, 3, 3)
+    ids = np.array([2, 0, 1], np.int32)
+    op = O.OraclePool(3, bits, 3)
+    op.load_fp32(ids, st)
+    gp = S.Pool(3, bits, 3, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    load_bytes(gp, ids, op.slot_bytes(ids))
+    out = torch.empty((3, 3, 128, 128), dtype=torch.float32, device="cuda")
+    gp.dump_fp32(slots_t(ids), out)
+    assert np.array_equal(out.cpu().numpy(), op.dump_fp32(ids))
+
+
+def test_packed_round_trip_bit_exact(S):
+    rng = np.random.default_rng(3)
+    bits = [6, 8, 4, 6]
+    gp = S.Pool(16, bits, 2)
+    stride = gp.slot_stride
+    data = rng.integers(0, 256, (5, stride), dtype=np.uint8)
+    ids = np.array([15, 3, 9, 0, 4], np.int32)
+    load_bytes(gp, ids, data)
+    assert np.array_equal(dump_bytes(gp, ids), data)
+    assert np.array_equal(dump_bytes(gp, [15]), data[:1])
+
+
+# --------------------------------------------------------------------------- hand-computed cases
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+def test_rank1_worked_case_on_gpu(S, bits):
+    g = json.load(open(os.path.join(GOLDEN, "rank1_worked_case.json")))["step1"]
+    gp = S.Pool(2, [bits], 1, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    k = np.zeros((2, 1, 128), f32)
+    k[:, 0, g["key_index"]] = 1
+    v = np.zeros((2, 1, 128), f32)
+    v[:, 0, :4] = g["v_head"]
+    q = np.random.default_rng(4).standard_normal((2, 1, 128)).astype(f32)
+    y = torch.empty((2, 1, 128), device="cuda")
+    gp.decode_step(slots_t([1, 0]), dev(q), dev(k), dev(v), dev(np.full((2, 1), g["alpha"], f32)),
+                   dev(np.full((2, 1), g["beta"], f32)), y)
+    raw = dump_bytes(gp, [1, 0])
+    for s in range(2):
+        Q, r, c = O.split_block(raw[s], bits)
+        assert list(Q[0, :4]) == g["codes_row0_head"][str(bits)]
+        assert not Q[1:].any() and not Q[0, 4:].any()
+        np.testing.assert_allclose(c[:4], g["c_head"], rtol=1e-6)
+        assert r[0] == pytest.approx(g["r0"][str(bits)], rel=1e-6) and not r[1:].any()
+    yh = y.cpu().numpy()
+    np.testing.assert_allclose(yh[:, 0], q[:, 0, :1] * v[:, 0], rtol=1e-6, atol=1e-12)
+
+
+def test_power_of_two_fade_equivariance_on_gpu(S):
+    rng = np.random.default_rng(5)
+    bits = [4, 6, 8]
+    st = random_states(rng, 2, 3)
+    op = O.OraclePool(2, bits, 3)
+    op.load_fp32(np.arange(2, dtype=np.int32), st)
+    outs = []
+    for alpha in (1.0, 0.25):
+        gp = S.Pool(2, bits, 3, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+        load_bytes(gp, [0, 1], op.slot_bytes([0, 1]))
+        z = np.zeros((2, 3, 128), f32)
+        y = torch.empty((2, 3, 128), device="cuda")
+        gp.decode_step(slots_t([0, 1]), dev(z), dev(z), dev(z), dev(np.full((2, 3), alpha, f32)),
+                       dev(np.zeros((2, 3), f32)), y)
+        outs.append(dump_bytes(gp, [0, 1]))
+    for s in range(2):
+        for h, b in enumerate(bits):
+            off, _ = O.head_offsets(bits)
+            n = O.block_bytes(b)
+            A = O.split_block(outs[0][s, off[h]:off[h] + n], b)
+            B = O.split_block(outs[1][s, off[h]:off[h] + n], b)
+            assert np.array_equal(A[0], B[0])
+            assert np.array_equal(A[1] / 2, B[1]) and np.array_equal(A[2] / 2, B[2])
+
+
+def _run_gpu(S, bits, Hk, gate, dtype, x, init_bytes, ids, num_slots):
+    gp = S.Pool(num_slots, bits, Hk, gate, dtype)
+    load_bytes(gp, ids, init_bytes)
+    tx = {}
+    for key, val in x.items():
+        if dtype == S.STEPQ_DTYPE_BF16:
+            tx[key] = dev(W.to_bf16_bits(val).view(np.int16))
+        else:
+            tx[key] = dev(val)
+    y = torch.empty(x["v"].shape, device="cuda")
+    gp.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    return y.cpu().numpy(), dump_bytes(gp, ids), gp.get_error()
+
+
+def test_kda_equal_gates_gqa_and_bf16_identities(S):
+    """Bit identities on the GPU: KDA with equal per-channel gates = GDN; Hk = 2 with
+    H = 4 = repeated key heads; bf16 inputs = the same values given as fp32."""
+    rng = np.random.default_rng(6)
+    bits = [4, 6, 8, 6]
+    n, H = 3, 4
+    op = O.OraclePool(4, bits, H)
+    ids = np.array([3, 1, 0], np.int32)
+    op.load_fp32(ids, random_states(rng, n, H))
+    init = op.slot_bytes(ids)
+    q2 = W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)]))
+    k2 = W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)]))
+    v = W.round_bf16(rng.standard_normal((n, H, 128)).astype(f32))
+    a = W.round_bf16(rng.uniform(0.5, 1, (n, H)).astype(f32))
+    b = W.round_bf16(rng.uniform(0, 1, (n, H)).astype(f32))
+    base = dict(q=q2, k=k2, v=v, alpha=a, beta=b)
+    y0, s0, e0 = _run_gpu(S, bits, 2, 0, S.STEPQ_DTYPE_F32, base, init, ids, 4)
+    rep = dict(base, q=np.repeat(q2, 2, 1), k=np.repeat(k2, 2, 1))
+    y1, s1, e1 = _run_gpu(S, bits, 4, 0, S.STEPQ_DTYPE_F32, rep, init, ids, 4)
+    kda = dict(base, alpha=np.repeat(a[:, :, None], 128, 2))
+    y2, s2, e2 = _run_gpu(S, bits, 2, 1, S.STEPQ_DTYPE_F32, kda, init, ids, 4)
+    y3, s3, e3 = _run_gpu(S, bits, 2, 0, S.STEPQ_DTYPE_BF16, base, init, ids, 4)
+    assert e0 == e1 == e2 == e3 == 0
+    for yy, ss in ((y1, s1), (y2, s2), (y3, s3)):
+        assert np.array_equal(yy, y0)
+        assert np.array_equal(ss, s0)
+
+
+def test_slot_permutation_invariance_and_bad_slot(S):
+    """The same requests placed in other slots give bit-identical results; an
+    out-of-range slot id raises the device flag, is skipped, and leaves the others intact."""
+    rng = np.random.default_rng(7)
+    bits = [6, 8]
+    n, H = 4, 2
+    states = random_states(rng, n, H)
+    op = O.OraclePool(n, bits, H)
+    op.load_fp32(np.arange(n, dtype=np.int32), states)
+    per_req = op.slot_bytes(np.arange(n))
+    x = dict(q=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+             k=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.8, 1, (n, H)).astype(f32), beta=rng.uniform(0, 1, (n, H)).astype(f32))
+    ya, sa, ea = _run_gpu(S, bits, H, 0, S.STEPQ_DTYPE_F32, x, per_req, np.array([0, 1, 2, 3], np.int32), 8)
+    yb, sb, eb = _run_gpu(S, bits, H, 0, S.STEPQ_DTYPE_F32, x, per_req, np.array([6, 2, 7, 0], np.int32), 8)
+    assert ea == eb == 0
+    assert np.array_equal(ya, yb) and np.array_equal(sa, sb)
+    # bad slot: request 2 points outside the pool
+    gp = S.Pool(8, bits, H, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    load_bytes(gp, [0, 1, 3], per_req[[0, 1, 3]])
+    y = torch.full((n, H, 128), 7.0, device="cuda")
+    tx = {k_: dev(v_) for k_, v_ in x.items()}
+    gp.decode_step(slots_t([0, 1, 99, 3]), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    assert gp.get_error() == S.STEPQ_FLAG_BAD_SLOT
+    assert gp.get_error() == 0                        # reading clears the flag
+    yh = y.cpu().numpy()
+    assert np.array_equal(yh[[0, 1, 3]], ya[[0, 1, 3]])
+    assert np.all(yh[2] == 7.0)                       # skipped request: y untouched
+    assert np.array_equal(dump_bytes(gp, [0, 1, 3]), sa[[0, 1, 3]])
+
+
+def test_zero_requests_and_invalid_arguments(S):
+    gp = S.Pool(4, [4, 8], 1)
+    empty = torch.empty(0, dtype=torch.int32, device="cuda")
+    t = torch.zeros(16, device="cuda")
+    gp.decode_step(empty, t, t, t, t, t, t)           # n = 0: no-op
+    lib = S.load_library()
+    assert lib.stepq_decode_step(gp.handle, None, 1, None, None, None, None, None, None, None) == -1
+    assert lib.stepq_pool_load_fp32(gp.handle, slots_t([0]).data_ptr(), 1, None, None) == -1
+    with pytest.raises(S.StepqError):
+        S.stepq_pool_create(4, [4, 5], 1)             # unsupported width
+    with pytest.raises(S.StepqError):
+        S.stepq_pool_create(4, [4, 8], 3)             # key heads must divide value heads
+    assert gp.get_error() == 0
+
+
+# --------------------------------------------------------------------------- workload parity
+
+CASES = [
+    # (config, variant, batch, layer, sampled requests, steps compared)
+    (1, "mixed6", None, 0, 4, 16),
+    (2, "mixed6", None, 0, 8, 64),
+    (3, "mixed6", None, 0, 6, 64),
+    (4, "mixed6", None, 0, 6, 64),
+    (4, "uniform4", None, 0, 6, 32),
+    (5, "mixed6", 64, 17, 3, 32),
+    (5, "mixed6", 256, 17, 3, 32),
+    (5, "mixed6", 1024, 0, 3, 32),
+    (5, "mixed6", 1024, 35, 3, 32),
+]
+
+
+@pytest.mark.parametrize("config,variant,batch,layer,nsample,steps", CASES,
+                         ids=["cfg%d-%s-b%s-l%d" % (c[0], c[1], c[2], c[3]) for c in CASES])
+def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
+    """Full batch on the GPU (the launch configuration of the benchmark); the oracle
+    follows a seeded sample of requests.  Every step: single-step tolerances (codes +-1
+    at rate <= 1e-5, r/c ulps, y max-rel <= 1e-4).  Whole trajectory: y relative L2 <= 1e-3.
+    A state whose codes came out +-1 from the oracle's is re-synchronised from the
+    oracle's bytes before the next step (oracle -> GPU only): a single such flip is
+    amplified by the recurrence itself, so free-running trajectories are not comparable."""
+    w = W.make_workload(config, variant, batch)
+    bits = PH.head_bits(w, layer)
+    sub = W.sample_requests(w, nsample)
+    sub_slots = w.slot_ids[sub]
+    op = PH.oracle_pool_with_warmup(w, bits, sub, layer)
+    gp = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    load_bytes(gp, sub_slots, op.slot_bytes(sub_slots))
+    all_slots = slots_t(w.slot_ids)
+    num = den = 0.0
+    flips = elements = resyncs = 0
+    worst = dict(max_code_diff=0, r_ulp=0, c_ulp=0, y=0.0)
+    for t in range(steps):
+        x = W.step_inputs(w, t, W.PHASE_RUN, layer)
+        tx = PH.to_device(w, x, torch)
+        y = torch.empty((w.B, w.H, w.dv), device="cuda")
+        gp.decode_step(all_slots, tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        xs = PH.sub_inputs(x, sub)
+        yo = op.decode_step(sub_slots, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"])
+        yg = y[torch.from_numpy(sub).cuda()].cpu().numpy()
+        num += float(np.sum((yg.astype(np.float64) - yo) ** 2))
+        den += float(np.sum(yo.astype(np.float64) ** 2))
+        worst["y"] = max(worst["y"], PH.y_max_rel(yg, yo))
+        gb, ob = dump_bytes(gp, sub_slots), op.slot_bytes(sub_slots)
+        res = PH.compare_slots(gb, ob, bits)
+        flips += res["flips"]
+        elements += res["elements"]
+        for key in ("max_code_diff", "r_ulp", "c_ulp"):
+            worst[key] = max(worst[key], res[key])
+        if not res["byte_equal"]:
+            load_bytes(gp, sub_slots, ob)
+            resyncs += 1
+    assert gp.get_error() == 0
+    rel = np.sqrt(num / den)
+    print("\n%s: y rel L2 %.3e, worst %s, flips %d / %d (%.2e), resyncs %d" %
+          (w.name, rel, worst, flips, elements, flips / elements, resyncs))
+    assert worst["max_code_diff"] <= 1
+    assert flips <= PH.CODE_FLIP_RATE * elements
+    assert worst["r_ulp"] <= PH.R_ULP and worst["c_ulp"] <= PH.C_ULP
+    assert worst["y"] <= PH.Y_MAX_REL
+    assert rel <= PH.Y_TRAJ_REL_L2
