@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--input-sets", type=int, default=N_INPUT_SETS,
+                    help="distinct per-step input batches kept on the device and cycled")
     return ap.parse_args()
 
 
@@ -243,7 +245,7 @@ def main():
     # per-step inputs, resident in HBM (bf16 bit patterns)
     def dev_inputs(x):
         return {k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).cuda() for k, v in x.items()}
-    nsets = min(N_INPUT_SETS, args.steps + args.warmup)
+    nsets = max(1, min(args.input_sets, args.steps + args.warmup))
     host_sets = [W.step_inputs(w, t) for t in range(nsets)]
     sets = [dev_inputs(x) for x in host_sets]
     y = torch.empty((w.B, w.H, w.dv), device="cuda")

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstepq.so")
-SOURCES = ["stepq_kernels.cu", "stepq_capi.cu", "stepq_alloc.cpp"]
+SOURCES = ["stepq_decode.cu", "stepq_io.cu", "stepq_capi.cu", "stepq_alloc.cpp"]
 HEADERS = ["stepq_device.cuh", "stepq_tile.cuh", "stepq_internal.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -1,6 +1,7 @@
 // stepq_capi.cu -- the C ABI of libstepq (declared in include/stepq.h): pool
 // management, argument validation and kernel launches.  Every step of the decode
-// path runs in the kernels of stepq_kernels.cu; this file only checks and launches.
+// path runs in the kernels of stepq_decode.cu and stepq_io.cu; this file only checks
+// arguments and launches.
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -44,6 +45,7 @@ void free_pool(stepq_pool *p)
     cudaFree(p->d_pool);
     cudaFree(p->d_offs);
     cudaFree(p->d_bits);
+    cudaFree(p->d_order);
     cudaFree(p->d_flag);
     delete p;
 }
@@ -101,11 +103,20 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     if (e == cudaSuccess) e = cudaMalloc(&p->d_pool, size_t(p->total));
     if (e == cudaSuccess) e = cudaMalloc(&p->d_offs, sizeof(long long) * p->H);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_bits, size_t(p->H));
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * p->H);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_flag, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(p->d_pool, 0, size_t(p->total));
     if (e == cudaSuccess) e = cudaMemset(p->d_flag, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemcpy(p->d_offs, p->offs.data(), sizeof(long long) * p->H, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_bits, p->bits.data(), size_t(p->H), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) {
+        // the decode kernel visits heads grouped by bit width (stable within a width)
+        std::vector<int32_t> order;
+        for (int w = 4; w <= 8; w += 2)
+            for (int h = 0; h < p->H; ++h)
+                if (p->bits[h] == w) order.push_back(h);
+        e = cudaMemcpy(p->d_order, order.data(), sizeof(int32_t) * p->H, cudaMemcpyHostToDevice);
+    }
     if (e == cudaSuccess) e = stepq::decode_configure(p);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {

@@ -1,0 +1,569 @@
+// stepq_decode.cu -- the fused decode step of the quantized gated Delta-rule layer (sm_100a).
+//
+// Per (request b, value head h) state, one pass (STEPQuant summary, "Method": update the
+// reconstructed state in floating point, compute the output, then quantize for storage;
+// "Paper Explained", "The mechanism: rewriting state with the delta rule"):
+//   S'_ij = alpha_i r_i c_j Q_ij            dequantize + fade
+//   u_j   = sum_i S'_ij k_i                 predict (what the key currently retrieves)
+//   d_j   = beta (v_j - u_j)                write strength times the difference
+//   S_ij  = S'_ij + k_i d_j                 Delta write
+//   y_j   = sum_i S_ij q_i                  readout from the updated, unquantized state
+//   c_j   = sqrt(max_i |S_ij|),  r_i = max_j (|S_ij| / c_j) / qmax      clip-free refit
+//   Q_ij  = round-half-even(S_ij / (r_i c_j)), repacked in place
+//
+// Arithmetic: with rho_i = alpha_i r_i, both column dot products run on the integer codes
+// with per-row weights (u_j = c_j sum_i Q_ij rho_i k_i, y'_j = c_j sum_i Q_ij rho_i q_i,
+// y_j = y'_j + (k.q) d_j), and the updated state is kept column-scaled:
+// S_ij = c_j T_ij with T_ij = rho_i Q_ij + k_i (d_j / c_j).  The refit then needs
+// max_i |T_ij|, the new column factor, and P_ij = T_ij (c_j / c_new_j) = S_ij / c_new_j.
+//
+// Threads: 256 per state.  Warp w owns the 16-column panel w; lane l holds rows l + 32 m
+// (m = 0..3) of it: 64 state values in registers.  Column sums and maxima reduce over the
+// warp's lanes.  Row maxima over the 8 panels go through shared memory, where thread t
+// (t < 128) finalizes row t (r_t and 1/r_t) while threads 128..255 build the per-row
+// weights of the next state, so every row-wise quantity is computed once.  Row weights
+// are stored as duplicated pairs, the operand form of the packed f32x2 instructions.
+//
+// Data movement: persistent CTAs; items are dealt round-robin in head-major order and the
+// heads are visited grouped by bit width, so the CTAs resident at a time share one code
+// path.  Thread 0 bulk-copies the packed head block and q, k, v (and the KDA gate) of item
+// i+2 into a 4-stage shared-memory ring while the CTA computes item i (full barriers:
+// mbarrier transaction counts; empty barriers: one arrival per warp once its stores have
+// read the stage).  After the refit each warp bulk-stores its panel and its slice of c
+// from the stage (warp 0 also r).  Each state is read from HBM once and written once.
+#include <cfloat>
+#include <cstdint>
+
+#include "stepq_internal.h"
+#include "stepq_tile.cuh"
+
+namespace stepq {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kIoBytes = 512;       // stage room for one 128-vector input (fp32 or bf16)
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRows = 4;            // rows per thread
+constexpr int kRpStride = 12;       // padded row stride of the row-maxima exchange (floats)
+constexpr unsigned kFull = 0xffffffffu;
+
+struct StageMeta {
+    long long dst;                  // byte offset of the head block in the pool
+    int valid;
+    int bits;
+};
+
+struct DecodeArgs {
+    uint8_t *pool;
+    long long slot_stride;
+    const long long *head_off;
+    const uint8_t *head_bits;
+    const int32_t *head_order;      // processing order of the heads (grouped by bit width)
+    int num_slots, H, Hk, group;
+    const int32_t *slot_ids;
+    int n;
+    int step_b, step_h;             // gridDim.x in head-major items = step_h * n + step_b
+    const void *q, *k, *v, *alpha, *beta;
+    float *y;
+    int *flag;
+    int blk_cap, stage_bytes;
+};
+
+// Shared memory besides the ring.
+struct Scratch {
+    float rp[DK * kRpStride];       // row maxima of |P| per panel
+    float4 wlo[DK];                 // per row {rho k, rho k, rho q, rho q}  (lanes 0..15)
+    float4 whi[DK];                 // per row {rho q, rho q, rho k, rho k}  (lanes 16..31)
+    float4 wrk[DK];                 // per row {rho, rho, k, k}
+    float2 ir[DK];                  // per row {1/r, 1/r}
+    float xd[NPANEL * PANEL];       // d_j / c'_j per column
+    float xg[NPANEL * PANEL];       // c'_j / c_new_j per column
+    float kqw[4];                   // partial k.q of the next state (warps 4..7)
+    float invpos[3][PANEL];         // 1 / position scale of the unpacked field (bits 4, 6, 8)
+    long long hoff[kMaxHeads];      // head block offsets inside a slot
+    int32_t hord[kMaxHeads];        // head processing order
+    uint8_t hbits[kMaxHeads];       // head widths
+    StageMeta meta[kStages];
+    int prod_b, prod_h;             // producer cursor
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+};
+
+// 1 / (power-of-two scale of the unpacked field) by bit width and column in the panel
+__constant__ float kInvPos[3][PANEL];
+
+// Item cursor in head-major order (index = h * n + b), stepping by the grid size.
+struct Cursor {
+    int b, h;
+    __device__ __forceinline__ void advance(const DecodeArgs &a)
+    {
+        b += a.step_b;
+        h += a.step_h;
+        if (b >= a.n) { b -= a.n; ++h; }
+    }
+};
+
+// Per-row weights of a state held in a stage, built by thread t (128 <= t < 256) for row
+// t - 128, and the share of k.q of warps 4..7.
+template <int GATE, typename TIn>
+__device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs &a, int bits, float alpha_s,
+                                          Scratch &sc, int t)
+{
+    const int i = t - 128;
+    const float *r = reinterpret_cast<const float *>(stage + codes_bytes(bits));
+    const TIn *qs = reinterpret_cast<const TIn *>(stage + a.blk_cap);
+    const TIn *ks = reinterpret_cast<const TIn *>(stage + a.blk_cap + kIoBytes);
+    const TIn *as = reinterpret_cast<const TIn *>(stage + a.blk_cap + 3 * kIoBytes);
+    const float al = (GATE == STEPQ_GATE_KDA) ? to_f32(as[i]) : alpha_s;
+    const float rho = al * r[i];
+    const float k = to_f32(ks[i]);
+    const float q = to_f32(qs[i]);
+    const float rk = rho * k, rq = rho * q;
+    sc.wlo[i] = make_float4(rk, rk, rq, rq);
+    sc.whi[i] = make_float4(rq, rq, rk, rk);
+    sc.wrk[i] = make_float4(rho, rho, k, k);
+    float kq = k * q;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
+    if ((t & 31) == 0) sc.kqw[(t >> 5) - 4] = kq;
+}
+
+// One state: the register tile through the row-maxima exchange, the row finalization /
+// next row table, then quantization, packing and the per-warp stores.  Returns false on
+// every thread when some thread saw a failed wait.
+template <int GATE, typename TIn, int BITS>
+__device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_next, const DecodeArgs &a, Scratch &sc,
+                                            const TileIdx<4> &ix, int tid, long long bh, float beta, float kq,
+                                            TIn alpha_next_raw, bool ok)
+{
+    uint8_t *stage = stages + (i % kStages) * a.stage_bytes;
+    constexpr int QM = qmax_of(BITS);
+    constexpr float MAG = kTwo23 + float(1 << (BITS - 1));
+    constexpr int BI = BITS == 4 ? 0 : BITS == 6 ? 1 : 2;
+    const int lane = ix.lane;
+    const int panel = ix.panel;
+    const bool upper = (lane & 16) != 0;            // lanes holding the q-weighted sums first
+    const int col = lane & 15;                      // the column this lane finalizes
+
+    uint8_t *codes = stage;
+    float *r_io = reinterpret_cast<float *>(stage + codes_bytes(BITS));
+    float *c_io = r_io + DK;
+    const TIn *vs = reinterpret_cast<const TIn *>(stage + a.blk_cap + 2 * kIoBytes);
+
+    // ---- codes of the thread's 4 rows x 16 columns (times their position scale), exact floats
+    float T[kRows][PANEL];
+#pragma unroll
+    for (int m = 0; m < kRows; ++m)
+        load_codes<BITS>(codes + panel * panel_bytes(BITS) + ix.row(m) * seg_bytes(BITS), T[m]);
+
+    // A zero column factor means a zero column whatever its codes (a fresh pool holds
+    // nonzero codes under zero scales): clear those codes.  Warp-uniform and rare.
+    const float cj = c_io[panel * PANEL + col];
+    if (__any_sync(kFull, cj == 0.0f)) {
+#pragma unroll
+        for (int j = 0; j < PANEL; ++j) {
+            const float z = c_io[panel * PANEL + j] == 0.0f ? 0.0f : 1.0f;
+#pragma unroll
+            for (int m = 0; m < kRows; ++m) T[m][j] *= z;
+        }
+    }
+    // column factor of the scaled codes (a zero column behaves as c = 1: S = T = k d)
+    const float cprime = (cj == 0.0f ? 1.0f : cj) * sc.invpos[BI][col];
+
+    // ---- column dot products over the thread's rows (column pairs, f32x2), then over the
+    // warp: lane bit 4 first (select-free: the partner's second sum is this lane's first
+    // quantity), then bits 3..0.  Lanes 0..15 end with u_col, lanes 16..31 with y'_col.
+    const float4 *wt = upper ? sc.whi : sc.wlo;
+    float4 w[kRows];
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) w[m] = wt[ix.row(m)];
+    float A[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 2) {
+        float2 s1 = fmul2(make_float2(T[0][j], T[0][j + 1]), make_float2(w[0].x, w[0].y));
+        float2 s2 = fmul2(make_float2(T[0][j], T[0][j + 1]), make_float2(w[0].z, w[0].w));
+#pragma unroll
+        for (int m = 1; m < kRows; ++m) {
+            s1 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].x, w[m].y), s1);
+            s2 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].z, w[m].w), s2);
+        }
+        A[j] = s1.x + __shfl_xor_sync(kFull, s2.x, 16);
+        A[j + 1] = s1.y + __shfl_xor_sync(kFull, s2.y, 16);
+    }
+    reduce_scatter<PANEL, 4, 8, false>(A, lane);
+
+    // d_j = beta (v_j - u_j) (lanes 0..15); y_j = y'_j + (k.q) d_j (lanes 16..31)
+    const float val = cprime * A[0];
+    const float delta = beta * (to_f32(vs[panel * PANEL + col]) - val);
+    const float dpair = __shfl_xor_sync(kFull, delta, 16);
+    if (upper)
+        a.y[bh * DV + panel * PANEL + col] = fmaf(dpair, kq, val);
+    else
+        sc.xd[panel * PANEL + col] = div_refined(delta, cprime);
+    __syncwarp();
+    float dd[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(sc.xd + panel * PANEL + j);
+        dd[j] = t.x; dd[j + 1] = t.y; dd[j + 2] = t.z; dd[j + 3] = t.w;
+    }
+
+    // ---- T_ij = rho_i Q_ij + k_i d'_j (the updated state is c'_j T_ij); column maxima of |T|
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+        const float4 rk = sc.wrk[ix.row(m)];
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            float2 t = fmul2(make_float2(T[m][j], T[m][j + 1]), make_float2(rk.x, rk.y));
+            t = ffma2(make_float2(rk.z, rk.w), make_float2(dd[j], dd[j + 1]), t);
+            T[m][j] = t.x;
+            T[m][j + 1] = t.y;
+        }
+    }
+    // column maxima: over the thread's rows, then a warp-wide max per column; the 16
+    // results go through shared memory (the d' buffer, already read) to the column lanes
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        float cm[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            cm[e] = warp_absmax(fmaxf(absmax3(T[0][j + e], T[1][j + e], T[2][j + e]), fabsf(T[3][j + e])));
+        if (lane == 0)
+            *reinterpret_cast<float4 *>(sc.xd + panel * PANEL + j) = make_float4(cm[0], cm[1], cm[2], cm[3]);
+    }
+    __syncwarp();
+    const float tmax = sc.xd[panel * PANEL + col];
+
+    // c_new = sqrt(max_i |S_ij|); the scaled state divides by it: g_j = c'_j / c_new_j
+    const float cnew = sqrt_refined(cprime * tmax);
+    const float g = cnew > 0.0f ? div_refined(cprime, cnew) : 0.0f;
+    if (!upper) {
+        c_io[panel * PANEL + col] = cnew;
+        sc.xg[panel * PANEL + col] = g;
+    }
+    __syncwarp();
+    float gg[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(sc.xg + panel * PANEL + j);
+        gg[j] = t.x; gg[j + 1] = t.y; gg[j + 2] = t.z; gg[j + 3] = t.w;
+    }
+    // P_ij = S_ij / c_new_j and the thread's row maxima of |P| (panel partials)
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            const float2 p = fmul2(make_float2(T[m][j], T[m][j + 1]), make_float2(gg[j], gg[j + 1]));
+            T[m][j] = p.x;
+            T[m][j + 1] = p.y;
+        }
+        float mx = absmax3(T[m][0], T[m][1], T[m][2]);
+#pragma unroll
+        for (int j = 3; j < PANEL - 1; j += 2) mx = absmax3(mx, T[m][j], T[m][j + 1]);
+        mx = fmaxf(mx, fabsf(T[m][PANEL - 1]));
+        sc.rp[ix.row(m) * kRpStride + panel] = mx;
+    }
+    if (__syncthreads_or(!ok)) return false;
+
+    // ---- threads 0..127: r_t = max_j |P_tj| / qmax and 1 / r_t for row t;
+    //      threads 128..255: the next state's row weights
+    bool tiny = false;
+    if (tid < DK) {
+        const float4 u = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride);
+        const float4 v = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride + 4);
+        const float mr = fmaxf(max3(u.x, u.y, u.z), max3(max3(u.w, v.x, v.y), v.z, v.w));
+        const float r = div_const<QM>(mr);
+        r_io[tid] = r;
+        tiny = r > 0.0f && r < FLT_MIN;
+        const float ir = r >= FLT_MIN ? rcp_refined(r) : 0.0f;
+        sc.ir[tid] = make_float2(ir, ir);
+    } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
+        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
+                             to_f32(alpha_next_raw), sc, tid);
+    }
+    const bool any_tiny = __syncthreads_or(tiny);
+
+    // ---- codes = round-half-even(P_ij / r_i): fma(P, 1/r, 2^23 + 2^(b-1)) rounds to the
+    // nearest integer, ties to even, leaving the offset-binary code in the low mantissa bits
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+        const int row = ix.row(m);
+        const float2 ir = sc.ir[row];
+        uint32_t u[PANEL];
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), ir, make_float2(MAG, MAG));
+            u[j] = __float_as_uint(f.x);
+            u[j + 1] = __float_as_uint(f.y);
+        }
+        if (any_tiny) {
+            // subnormal row factor: 1/r overflows; divide element by element
+            const float r = r_io[row];
+            if (r > 0.0f && r < FLT_MIN) {
+#pragma unroll
+                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(__fdiv_rn(T[m][j], r) + MAG);
+            }
+        }
+        pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
+    }
+    // each warp stores its panel of codes and its slice of c (warp 0 also r)
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        uint8_t *dst = a.pool + sc.meta[i % kStages].dst;
+        bulk_s2g(dst + panel * panel_bytes(BITS), codes + panel * panel_bytes(BITS), panel_bytes(BITS));
+        bulk_s2g(dst + codes_bytes(BITS) + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
+        if (panel == 0) bulk_s2g(dst + codes_bytes(BITS), r_io, 4 * DK);
+    }
+    return true;
+}
+
+template <int GATE, typename TIn>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *stages = smem;
+    Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * a.stage_bytes);
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const long long total = (long long)a.n * a.H;
+    const long long first = blockIdx.x;
+    if (first >= total) return;
+    const int count = int((total - first + gridDim.x - 1) / gridDim.x);
+    constexpr int esz = sizeof(TIn);
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sc.full[s], 1);
+            mbar_init(&sc.empty[s], kWarps);
+        }
+        fence_mbarrier_init();
+    }
+    if (tid < 3 * PANEL) sc.invpos[tid / PANEL][tid % PANEL] = kInvPos[tid / PANEL][tid % PANEL];
+    for (int h = tid; h < a.H; h += kThreads) {
+        sc.hoff[h] = a.head_off[h];
+        sc.hord[h] = a.head_order[h];
+        sc.hbits[h] = a.head_bits[h];
+    }
+    __syncthreads();
+
+    const Cursor start = {int(first % a.n), int(first / a.n)};
+
+    // ---- producer (thread 0): bulk-copy item j's inputs into stage j % kStages
+    int slot_next = 0;                  // producer: prefetched slot id of the next item to issue
+    auto issue = [&](int j) {
+        const int st = j % kStages;
+        const int slot = slot_next;
+        Cursor pc = {sc.prod_b, sc.prod_h};
+        const int b = pc.b, h = sc.hord[pc.h], g = h / a.group;
+        pc.advance(a);
+        sc.prod_b = pc.b;
+        sc.prod_h = pc.h;
+        if (j + 1 < count) slot_next = __ldg(a.slot_ids + pc.b);
+        uint8_t *stage = stages + st * a.stage_bytes;
+        StageMeta &mt = sc.meta[st];
+        if (slot < 0 || slot >= a.num_slots) {
+            mt.valid = 0;
+            atomicOr(a.flag, STEPQ_FLAG_BAD_SLOT);
+            mbar_arrive(&sc.full[st]);
+        } else {
+            const int bits = sc.hbits[h];
+            const uint32_t bb = uint32_t(block_bytes(bits));
+            const long long bh = (long long)b * a.H + h;
+            const long long kqrow = (long long)b * a.Hk + g;
+            mt.valid = 1;
+            mt.bits = bits;
+            mt.dst = (long long)slot * a.slot_stride + sc.hoff[h];
+            const uint32_t io = DK * esz;
+            mbar_arrive_expect_tx(&sc.full[st], bb + 3 * io + (GATE == STEPQ_GATE_KDA ? io : 0u));
+            bulk_g2s(stage, a.pool + mt.dst, bb, &sc.full[st]);
+            bulk_g2s(stage + a.blk_cap, static_cast<const uint8_t *>(a.q) + kqrow * io, io, &sc.full[st]);
+            bulk_g2s(stage + a.blk_cap + kIoBytes, static_cast<const uint8_t *>(a.k) + kqrow * io, io, &sc.full[st]);
+            bulk_g2s(stage + a.blk_cap + 2 * kIoBytes, static_cast<const uint8_t *>(a.v) + bh * io, io, &sc.full[st]);
+            if (GATE == STEPQ_GATE_KDA)
+                bulk_g2s(stage + a.blk_cap + 3 * kIoBytes, static_cast<const uint8_t *>(a.alpha) + bh * io, io,
+                         &sc.full[st]);
+        }
+    };
+    if (tid == 0) {
+        sc.prod_b = start.b;
+        sc.prod_h = start.h;
+        slot_next = __ldg(a.slot_ids + start.b);
+        issue(0);
+        if (count > 1) issue(1);
+    }
+
+    const TileIdx<4> ix(tid);
+    const TIn *alpha_g = static_cast<const TIn *>(a.alpha);
+    const TIn *beta_g = static_cast<const TIn *>(a.beta);
+
+    // ---- prologue: the first state's row table
+    Cursor cur = start;
+    long long bh_cur = (long long)cur.b * a.H + sc.hord[cur.h];
+    float beta_cur = to_f32(beta_g[bh_cur]);
+    bool ok = mbar_wait_bounded(&sc.full[0], 0u);
+    {
+        const StageMeta m0 = sc.meta[0];
+        const float al0 = (GATE == STEPQ_GATE_GDN) ? to_f32(alpha_g[bh_cur]) : 1.0f;
+        if (m0.valid && tid >= DK) row_table<GATE, TIn>(stages, a, m0.bits, al0, sc, tid);
+    }
+    __syncthreads();
+
+    int aborted_at = -1;
+    for (int i = 0; i < count; ++i) {
+        const int st = i % kStages;
+        if (lane == 0 && i >= 2) {
+            bulk_wait_read<1>();                      // this warp's stores of item i-2 have read their stage
+            mbar_arrive(&sc.empty[(i - 2) % kStages]);
+        }
+        if (tid == 0 && i + 2 < count) {
+            if (i + 2 >= kStages)                    // stage (i+2)%4 last held item i-2
+                ok &= mbar_wait_bounded(&sc.empty[(i + 2) % kStages], uint32_t((i - 2) / kStages) & 1u);
+            issue(i + 2);
+        }
+        // next item: cursor, scalar gates, its stage (waited for before its row table is built)
+        Cursor nxt = cur;
+        nxt.advance(a);
+        const bool has_next = i + 1 < count;
+        const long long bh_next = has_next ? (long long)nxt.b * a.H + sc.hord[nxt.h] : 0;
+        TIn beta_raw = TIn(0), alpha_raw = TIn(0);            // converted when used
+        if (has_next) {
+            beta_raw = beta_g[bh_next];
+            if (GATE == STEPQ_GATE_GDN) alpha_raw = alpha_g[bh_next];
+        }
+        const float4 kqv = *reinterpret_cast<const float4 *>(sc.kqw);
+        const float kq = (kqv.x + kqv.y) + (kqv.z + kqv.w);
+        const int valid = sc.meta[st].valid, bits = sc.meta[st].bits;
+        if (has_next) ok &= mbar_wait_bounded(&sc.full[(i + 1) % kStages], uint32_t((i + 1) / kStages) & 1u);
+        bool alive;
+        if (!valid) {
+            alive = !__syncthreads_or(!ok);
+            if (alive) {
+                const StageMeta mn = sc.meta[(i + 1) % kStages];
+                if (has_next && mn.valid && tid >= DK)
+                    row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits, to_f32(alpha_raw),
+                                         sc, tid);
+                __syncthreads();
+            }
+        } else if (bits == 4) {
+            alive = decode_item<GATE, TIn, 4>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
+        } else if (bits == 6) {
+            alive = decode_item<GATE, TIn, 6>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
+        } else {
+            alive = decode_item<GATE, TIn, 8>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
+        }
+        if (!alive) {
+            aborted_at = i;
+            break;
+        }
+        if (lane == 0) bulk_commit();
+        cur = nxt;
+        bh_cur = bh_next;
+        beta_cur = to_f32(beta_raw);
+    }
+    if (lane == 0) bulk_wait_all();
+    if (tid == 0 && aborted_at >= 0) {
+        atomicOr(a.flag, STEPQ_FLAG_TIMEOUT);
+        // let the loads still in flight land before the CTA leaves (bounded waits)
+        const int issued = aborted_at + 2 < count ? aborted_at + 3 : count;
+        for (int j = aborted_at; j < issued; ++j)
+            (void)mbar_wait_bounded(&sc.full[j % kStages], uint32_t(j / kStages) & 1u);
+    }
+}
+
+size_t decode_smem_bytes(int stage_bytes)
+{
+    return size_t(kStages) * stage_bytes + sizeof(Scratch);
+}
+
+// Largest dynamic shared memory any pool can ask for: 8-bit blocks plus four input vectors.
+// Every instantiation is opened up to it once, so pools of different shapes can share it.
+size_t decode_smem_max()
+{
+    return decode_smem_bytes((block_bytes(8) + 4 * kIoBytes + 127) / 128 * 128);
+}
+
+template <int GATE, typename TIn>
+cudaError_t configure_one(stepq_pool *p)
+{
+    auto kern = decode_kernel<GATE, TIn>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, p->decode_smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    p->decode_grid = per_sm * p->num_sms;
+    return cudaSuccess;
+}
+
+cudaError_t upload_tables()
+{
+    float h[3][PANEL];
+    const int widths[3] = {4, 6, 8};
+    for (int b = 0; b < 3; ++b)
+        for (int p = 0; p < PANEL; ++p) h[b][p] = 1.0f / pos_scale(widths[b], p);
+    return cudaMemcpyToSymbol(kInvPos, h, sizeof(h));
+}
+
+}  // namespace
+
+cudaError_t decode_configure(stepq_pool *p)
+{
+    cudaError_t e = upload_tables();
+    if (e != cudaSuccess) return e;
+    p->blk_cap = p->max_block;
+    const int io = (p->gate_mode == STEPQ_GATE_KDA ? 4 : 3) * kIoBytes;
+    p->stage_bytes = (p->blk_cap + io + 127) / 128 * 128;
+    p->decode_smem = decode_smem_bytes(p->stage_bytes);
+    if (p->gate_mode == STEPQ_GATE_GDN)
+        return p->in_dtype == STEPQ_DTYPE_BF16 ? configure_one<STEPQ_GATE_GDN, uint16_t>(p)
+                                              : configure_one<STEPQ_GATE_GDN, float>(p);
+    return p->in_dtype == STEPQ_DTYPE_BF16 ? configure_one<STEPQ_GATE_KDA, uint16_t>(p)
+                                          : configure_one<STEPQ_GATE_KDA, float>(p);
+}
+
+cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, const void *q, const void *k,
+                          const void *v, const void *alpha, const void *beta, float *y, cudaStream_t stream)
+{
+    DecodeArgs a;
+    a.pool = p->d_pool;
+    a.slot_stride = p->slot_stride;
+    a.head_off = p->d_offs;
+    a.head_bits = p->d_bits;
+    a.head_order = p->d_order;
+    a.num_slots = p->num_slots;
+    a.H = p->H;
+    a.Hk = p->Hk;
+    a.group = p->H / p->Hk;
+    a.slot_ids = slot_ids;
+    a.n = n;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
+    a.y = y;
+    a.flag = p->d_flag;
+    a.blk_cap = p->blk_cap;
+    a.stage_bytes = p->stage_bytes;
+    // items are dealt round-robin in head-major order, so the CTAs resident at any moment
+    // work on one or two heads (one bit width: one code path in the instruction caches)
+    const long long total = (long long)n * p->H;
+    const int grid = int(total < p->decode_grid ? total : p->decode_grid);
+    a.step_b = grid % n;
+    a.step_h = grid / n;
+    if (p->gate_mode == STEPQ_GATE_GDN) {
+        if (p->in_dtype == STEPQ_DTYPE_BF16)
+            decode_kernel<STEPQ_GATE_GDN, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+        else
+            decode_kernel<STEPQ_GATE_GDN, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+    } else {
+        if (p->in_dtype == STEPQ_DTYPE_BF16)
+            decode_kernel<STEPQ_GATE_KDA, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+        else
+            decode_kernel<STEPQ_GATE_KDA, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace stepq

@@ -19,6 +19,7 @@ struct stepq_pool {
     uint8_t *d_pool = nullptr;          // [num_slots * slot_stride]
     long long *d_offs = nullptr;        // [H]
     uint8_t *d_bits = nullptr;          // [H]
+    int32_t *d_order = nullptr;         // [H] head processing order (grouped by bit width)
     int *d_flag = nullptr;              // sticky device flag (STEPQ_FLAG_* bits)
     int decode_grid = 0;                // persistent CTAs for the decode kernel
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel

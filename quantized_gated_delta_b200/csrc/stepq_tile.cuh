@@ -48,6 +48,15 @@ __host__ __device__ constexpr float pos_bias(int bits, int p)
 
 // ---------------------------------------------------------------- unpack one row segment
 
+// (a & mask) | magic in one three-input logic op; both constants are register operands
+// (a logic op encodes at most one immediate).
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t magic)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+    return d;
+}
+
 template <int BITS>
 __device__ __forceinline__ void unpack_seg(const uint8_t *seg, float (&f)[PANEL]);
 
@@ -71,14 +80,14 @@ __device__ __forceinline__ void unpack_seg<4>(const uint8_t *seg, float (&f)[PAN
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const uint32_t lo = ws[t], hi = ws[t] >> 16;
-        f[8 * t + 0] = __uint_as_float((lo & 0x0000Fu) | kMagicBits);
-        f[8 * t + 1] = __uint_as_float((lo & 0x000F0u) | kMagicBits);
-        f[8 * t + 2] = __uint_as_float((lo & 0x00F00u) | kMagicBits);
-        f[8 * t + 3] = __uint_as_float((lo & 0x0F000u) | kMagicBits);
-        f[8 * t + 4] = __uint_as_float((lo & 0xF0000u) | kMagicBits);
-        f[8 * t + 5] = __uint_as_float((hi & 0x000F0u) | kMagicBits);
-        f[8 * t + 6] = __uint_as_float((hi & 0x00F00u) | kMagicBits);
-        f[8 * t + 7] = __uint_as_float((hi & 0x0F000u) | kMagicBits);
+        f[8 * t + 0] = __uint_as_float(and_or(lo, 0x0000Fu, kMagicBits));
+        f[8 * t + 1] = __uint_as_float(and_or(lo, 0x000F0u, kMagicBits));
+        f[8 * t + 2] = __uint_as_float(and_or(lo, 0x00F00u, kMagicBits));
+        f[8 * t + 3] = __uint_as_float(and_or(lo, 0x0F000u, kMagicBits));
+        f[8 * t + 4] = __uint_as_float(and_or(lo, 0xF0000u, kMagicBits));
+        f[8 * t + 5] = __uint_as_float(and_or(hi, 0x000F0u, kMagicBits));
+        f[8 * t + 6] = __uint_as_float(and_or(hi, 0x00F00u, kMagicBits));
+        f[8 * t + 7] = __uint_as_float(and_or(hi, 0x0F000u, kMagicBits));
     }
 }
 
@@ -90,10 +99,10 @@ __device__ __forceinline__ void unpack_seg<6>(const uint8_t *seg, float (&f)[PAN
     const uint32_t g[4] = {w0, __funnelshift_r(w0, w1, 24), __funnelshift_r(w1, w2, 16), w2 >> 8};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        f[4 * k + 0] = __uint_as_float((g[k] & 0x0003Fu) | kMagicBits);
-        f[4 * k + 1] = __uint_as_float((g[k] & 0x00FC0u) | kMagicBits);
-        f[4 * k + 2] = __uint_as_float((g[k] & 0x3F000u) | kMagicBits);
-        f[4 * k + 3] = __uint_as_float(((g[k] >> 12) & 0x00FC0u) | kMagicBits);
+        f[4 * k + 0] = __uint_as_float(and_or(g[k], 0x0003Fu, kMagicBits));
+        f[4 * k + 1] = __uint_as_float(and_or(g[k], 0x00FC0u, kMagicBits));
+        f[4 * k + 2] = __uint_as_float(and_or(g[k], 0x3F000u, kMagicBits));
+        f[4 * k + 3] = __uint_as_float(and_or(g[k] >> 12, 0x00FC0u, kMagicBits));
     }
 }
 
