@@ -138,6 +138,30 @@ STEPQ_API int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32
                       const void *k, const void *v, const void *alpha, const void *beta, float *y,
                       stepq_stream stream);
 
+/* The decode step of stepq_decode_step for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point.  Some callers may not call cudaMalloc:
+ * code running inside a serving engine or framework that owns all device memory through
+ * its own arena or caching allocator (and accounts for every byte), or code embedded where
+ * new allocations are forbidden.  They keep the packed state themselves and pass it here;
+ * no pool object exists.
+ *   desc      as for stepq_pool_create (HOST, read during the call); num_heads <= 256, else
+ *             STEPQ_UNSUPPORTED (the scratch holds the tables of at most 256 heads)
+ *   state     DEVICE, caller-owned, 128-byte aligned: num_slots slots in the pool layout
+ *             (slot_stride = sum of the head block sizes), updated in place
+ *   slot_ids, q, k, v, alpha, beta, y   as for stepq_decode_step
+ *   flag_out  DEVICE, optional (may be NULL): receives this call's STEPQ_FLAG_* bits
+ * The kernel's scratch (the flag word and the per-head tables, 3328 bytes) is a fixed device
+ * array inside the library, held by every GPU that loads it until the process exits.  Every
+ * call rewrites it (flag cleared, tables refreshed) on `stream`; calls that overlap on the
+ * GPU (other streams, other threads) share it and race.  The first call on each device
+ * resolves the array's address and configures the kernel on that device, so it should come
+ * before any stream capture.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine). */
+STEPQ_API int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *state, const int32_t *slot_ids,
+                                        int32_t n, const void *q, const void *k, const void *v,
+                                        const void *alpha, const void *beta, float *y, int32_t *flag_out,
+                                        stepq_stream stream);
+
 /* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
  * Synchronizes the device. */
 STEPQ_API int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out);

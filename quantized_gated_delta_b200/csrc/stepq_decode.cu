@@ -567,3 +567,168 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
 }
 
 }  // namespace stepq
+
+// ------------------------------------------------------------------------------------------
+// stepq_decode_step_noalloc: the same decode kernel for callers that cannot allocate device
+// memory.  The caller brings the packed state buffer; the kernel's scratch (the sticky flag
+// word and the per-head tables that a pool keeps in its own allocations) lives in a
+// file-scope device array instead.
+// ------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace stepq {
+namespace {
+
+constexpr int kNoallocFlagOffset = 0;                                     // int32 flag word
+constexpr int kNoallocOffOffset = 256;                                    // int64[kMaxHeads]
+constexpr int kNoallocOrderOffset = kNoallocOffOffset + 8 * kMaxHeads;   // int32[kMaxHeads]
+constexpr int kNoallocBitsOffset = kNoallocOrderOffset + 4 * kMaxHeads;  // uint8[kMaxHeads]
+constexpr int kNoallocScratchBytes = kNoallocBitsOffset + kMaxHeads;      // 3328 bytes
+
+// Scratch of the allocation-free entry point.  Every GPU that loads the library holds it
+// until the process exits; host code reaches it only through the address returned by
+// cudaGetSymbolAddress (the symbol itself is a host-side stand-in).
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+struct NoallocDevice {
+    bool ready = false;
+    uint8_t *scratch = nullptr;         // device address of g_noalloc_scratch on this device
+    int num_sms = 0;
+};
+constexpr int kNoallocMaxDevices = 64;
+NoallocDevice g_noalloc_dev[kNoallocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Once per device, with that device current: resolve the scratch address and open the
+// kernel instantiations up to their largest shared-memory size.
+cudaError_t noalloc_setup(int dev, NoallocDevice **out)
+{
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoallocDevice &d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        void *ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = upload_tables();
+        if (e != cudaSuccess) return e;
+        const int smem = int(decode_smem_max());
+        e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        d.scratch = static_cast<uint8_t *>(ptr);
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
+template <int GATE, typename TIn>
+cudaError_t noalloc_launch(const DecodeArgs &a0, int num_sms, size_t smem, cudaStream_t stream)
+{
+    DecodeArgs a = a0;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<GATE, TIn>, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const long long total = (long long)a.n * a.H;
+    const long long cap = (long long)per_sm * num_sms;
+    const int grid = int(total < cap ? total : cap);
+    a.step_b = grid % a.n;
+    a.step_h = grid / a.n;
+    decode_kernel<GATE, TIn><<<grid, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace stepq
+
+extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *state, const int32_t *slot_ids,
+                                         int32_t n, const void *q, const void *k, const void *v, const void *alpha,
+                                         const void *beta, float *y, int32_t *flag_out, stepq_stream stream)
+{
+    using namespace stepq;
+    if (!desc || !desc->head_bits || n < 0) return STEPQ_INVALID_ARG;
+    if (desc->num_slots <= 0 || desc->num_heads <= 0 || desc->num_key_heads <= 0) return STEPQ_INVALID_ARG;
+    if (desc->num_heads % desc->num_key_heads != 0) return STEPQ_INVALID_ARG;
+    if (desc->num_heads > kMaxHeads) return STEPQ_UNSUPPORTED;       // scratch holds kMaxHeads heads
+    if (desc->gate_mode != STEPQ_GATE_GDN && desc->gate_mode != STEPQ_GATE_KDA) return STEPQ_INVALID_ARG;
+    if (desc->in_dtype != STEPQ_DTYPE_F32 && desc->in_dtype != STEPQ_DTYPE_BF16) return STEPQ_INVALID_ARG;
+    if (desc->d_k != DK || desc->d_v != DV) return STEPQ_UNSUPPORTED;
+    const int H = desc->num_heads;
+    for (int h = 0; h < H; ++h) {
+        const int b = desc->head_bits[h];
+        if (b != 4 && b != 6 && b != 8) return STEPQ_UNSUPPORTED;
+    }
+    if (n > desc->num_slots || n > 65535) return STEPQ_INVALID_ARG;
+    if (n == 0) return STEPQ_OK;
+    auto al = [](const void *p, uintptr_t m) { return (reinterpret_cast<uintptr_t>(p) & (m - 1)) == 0; };
+    const size_t esz = desc->in_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
+    if (!state || !slot_ids || !q || !k || !v || !alpha || !beta || !y) return STEPQ_INVALID_ARG;
+    if (!al(state, 128) || !al(slot_ids, 4) || !al(q, 16) || !al(k, 16) || !al(v, 16) || !al(y, 4) ||
+        !al(beta, esz) || !(desc->gate_mode == STEPQ_GATE_KDA ? al(alpha, 16) : al(alpha, esz)) ||
+        (flag_out && !al(flag_out, 4)))
+        return STEPQ_INVALID_ARG;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return STEPQ_CUDA_ERROR;
+    NoallocDevice *nd = nullptr;
+    if (noalloc_setup(dev, &nd) != cudaSuccess) return STEPQ_CUDA_ERROR;
+
+    // head tables (and a cleared flag word), staged in one host image of the scratch
+    alignas(16) uint8_t image[kNoallocScratchBytes] = {};
+    long long *off = reinterpret_cast<long long *>(image + kNoallocOffOffset);
+    int32_t *order = reinterpret_cast<int32_t *>(image + kNoallocOrderOffset);
+    uint8_t *bits = image + kNoallocBitsOffset;
+    long long stride = 0;
+    int max_block = 0, nord = 0;
+    for (int h = 0; h < H; ++h) {
+        off[h] = stride;
+        bits[h] = desc->head_bits[h];
+        stride += block_bytes(bits[h]);
+        if (block_bytes(bits[h]) > max_block) max_block = block_bytes(bits[h]);
+    }
+    for (int w = 4; w <= 8; w += 2)
+        for (int h = 0; h < H; ++h)
+            if (bits[h] == w) order[nord++] = h;
+    cudaError_t e = cudaMemcpyAsync(nd->scratch, image, kNoallocScratchBytes, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return STEPQ_CUDA_ERROR;
+
+    DecodeArgs a;
+    a.pool = state;
+    a.slot_stride = stride;
+    a.head_off = reinterpret_cast<const long long *>(nd->scratch + kNoallocOffOffset);
+    a.head_bits = nd->scratch + kNoallocBitsOffset;
+    a.head_order = reinterpret_cast<const int32_t *>(nd->scratch + kNoallocOrderOffset);
+    a.num_slots = desc->num_slots;
+    a.H = H;
+    a.Hk = desc->num_key_heads;
+    a.group = H / desc->num_key_heads;
+    a.slot_ids = slot_ids;
+    a.n = n;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
+    a.y = y;
+    a.flag = reinterpret_cast<int *>(nd->scratch + kNoallocFlagOffset);
+    a.blk_cap = max_block;
+    a.stage_bytes = (max_block + (desc->gate_mode == STEPQ_GATE_KDA ? 4 : 3) * kIoBytes + 127) / 128 * 128;
+    const size_t smem = decode_smem_bytes(a.stage_bytes);
+    if (desc->gate_mode == STEPQ_GATE_GDN)
+        e = desc->in_dtype == STEPQ_DTYPE_BF16 ? noalloc_launch<STEPQ_GATE_GDN, uint16_t>(a, nd->num_sms, smem, stream)
+                                               : noalloc_launch<STEPQ_GATE_GDN, float>(a, nd->num_sms, smem, stream);
+    else
+        e = desc->in_dtype == STEPQ_DTYPE_BF16 ? noalloc_launch<STEPQ_GATE_KDA, uint16_t>(a, nd->num_sms, smem, stream)
+                                               : noalloc_launch<STEPQ_GATE_KDA, float>(a, nd->num_sms, smem, stream);
+    if (e != cudaSuccess) return STEPQ_CUDA_ERROR;
+    if (flag_out) {
+        e = cudaMemcpyAsync(flag_out, nd->scratch + kNoallocFlagOffset, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            stream);
+        if (e != cudaSuccess) return STEPQ_CUDA_ERROR;
+    }
+    return STEPQ_OK;
+}

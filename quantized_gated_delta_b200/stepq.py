@@ -27,7 +27,7 @@ EXPORTED = [
     "stepq_pool_create", "stepq_pool_destroy", "stepq_pool_bytes", "stepq_pool_head_offset",
     "stepq_pool_load_fp32", "stepq_pool_load_packed", "stepq_pool_dump_fp32",
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
-    "stepq_allocate_bits", "stepq_status_string",
+    "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
 ]
 
 
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_decode_step": [P, P, I, P, P, P, P, P, P, P],
         "stepq_pool_get_error": [P, ctypes.POINTER(I)],
         "stepq_allocate_bits": [P, P, I, P, I, ctypes.c_double, P],
+        "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -156,6 +157,22 @@ def stepq_decode_step(pool: int, slot_ids, q, k, v, alpha, beta, y, stream=None)
     _check(load_library().stepq_decode_step(
         pool, _dev(slot_ids, "slot_ids"), slot_ids.numel(), _dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
         _dev(alpha, "alpha"), _dev(beta, "beta"), _dev(y, "y"), _stream(stream)), "stepq_decode_step")
+
+
+def stepq_decode_step_noalloc(num_slots: int, head_bits, num_key_heads: int, gate_mode: int, in_dtype: int,
+                              state, slot_ids, q, k, v, alpha, beta, y, flag_out=None, stream=None):
+    """Decode step on a caller-owned packed state buffer; the library allocates nothing.
+
+    For callers whose device memory all comes from their own allocator or arena (``state``
+    is such a buffer, in the pool layout).  ``flag_out``: optional int32 CUDA tensor that
+    receives the call's device flag bits."""
+    hb = np.ascontiguousarray(head_bits, dtype=np.uint8)
+    desc = stepq_pool_desc(int(num_slots), len(hb), int(num_key_heads), 128, 128, gate_mode, in_dtype,
+                           hb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    _check(load_library().stepq_decode_step_noalloc(
+        ctypes.byref(desc), _dev(state, "state"), _dev(slot_ids, "slot_ids"), slot_ids.numel(),
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(alpha, "alpha"), _dev(beta, "beta"), _dev(y, "y"),
+        None if flag_out is None else _dev(flag_out, "flag_out"), _stream(stream)), "stepq_decode_step_noalloc")
 
 
 def stepq_pool_get_error(pool: int) -> int:
