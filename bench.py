@@ -221,22 +221,17 @@ def main():
         run_reference(args)
         return
     import torch
-    import torch.distributed as dist
 
+    from quantized_gated_delta_b200 import dist as D
     from quantized_gated_delta_b200 import stepq
     from quantized_gated_delta_b200 import workloads as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    rank, world, local = D.init_from_env("nccl", timeout_s=120)
 
     w = W.make_workload(4, args.variant)
-    w.seed = w.seed + 1000 * rank                    # each rank serves its own requests
+    w.seed = D.shard_seed(w.seed, rank)              # each rank serves its own requests
     bits = w.head_bits[0] if w.head_bits is not None else stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
     bits = np.asarray(bits, dtype=np.uint8)
     pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
@@ -267,8 +262,7 @@ def main():
         sampler.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
+    D.barrier()
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
@@ -277,15 +271,10 @@ def main():
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    D.barrier()
     clocks = sampler.stop() if sampler else None
-    ms_total = t_start.elapsed_time(t_end)
+    ms_total = D.max_over_ranks(t_start.elapsed_time(t_end), "cuda")
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     err = pool.get_error()
     if err != 0:
         raise RuntimeError("device flag %d set during the timed region" % err)
@@ -318,19 +307,14 @@ def main():
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    D.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.e2e_steps):
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = D.max_over_ranks(e0.elapsed_time(e1), "cuda")
     e2e_value = units_per_step * args.e2e_steps * world / (ms_e2e / 1e3)
 
     base = None
@@ -363,8 +347,7 @@ def main():
         }
         print(json.dumps(line))
     pool.close()
-    if world > 1:
-        dist.destroy_process_group()
+    D.finalize()
 
 
 if __name__ == "__main__":
