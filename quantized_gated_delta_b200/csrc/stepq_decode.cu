@@ -62,6 +62,7 @@ struct DecodeArgs {
     const uint8_t *head_bits;
     const int32_t *head_order;      // processing order of the heads (grouped by bit width)
     int num_slots, H, Hk, group;
+    int nh4, nh6;                   // heads of width 4 and 6 (visited first, in that order)
     const int32_t *slot_ids;
     int n;
     int step_b, step_h;             // gridDim.x in head-major items = step_h * n + step_b
@@ -198,10 +199,8 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     const float val = cprime * A[0];
     const float delta = beta * (to_f32(vs[panel * PANEL + col]) - val);
     const float dpair = __shfl_xor_sync(kFull, delta, 16);
-    if (upper)
-        a.y[bh * DV + panel * PANEL + col] = fmaf(dpair, kq, val);
-    else
-        sc.xd[panel * PANEL + col] = div_refined(delta, cprime);
+    st_global_if(upper, a.y + bh * DV + panel * PANEL + col, fmaf(dpair, kq, val));
+    st_shared_if(!upper, sc.xd + panel * PANEL + col, div_refined(delta, cprime));
     __syncwarp();
     float dd[PANEL];
 #pragma unroll
@@ -230,8 +229,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
 #pragma unroll
         for (int e = 0; e < 4; ++e)
             cm[e] = warp_absmax(fmaxf(absmax3(T[0][j + e], T[1][j + e], T[2][j + e]), fabsf(T[3][j + e])));
-        if (lane == 0)
-            *reinterpret_cast<float4 *>(sc.xd + panel * PANEL + j) = make_float4(cm[0], cm[1], cm[2], cm[3]);
+        st_shared_v4_if(lane == 0, sc.xd + panel * PANEL + j, make_float4(cm[0], cm[1], cm[2], cm[3]));
     }
     __syncwarp();
     const float tmax = sc.xd[panel * PANEL + col];
@@ -239,10 +237,8 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     // c_new = sqrt(max_i |S_ij|); the scaled state divides by it: g_j = c'_j / c_new_j
     const float cnew = sqrt_refined(cprime * tmax);
     const float g = cnew > 0.0f ? div_refined(cprime, cnew) : 0.0f;
-    if (!upper) {
-        c_io[panel * PANEL + col] = cnew;
-        sc.xg[panel * PANEL + col] = g;
-    }
+    st_shared_if(!upper, c_io + panel * PANEL + col, cnew);
+    st_shared_if(!upper, sc.xg + panel * PANEL + col, g);
     __syncwarp();
     float gg[PANEL];
 #pragma unroll
@@ -299,11 +295,12 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
             u[j + 1] = __float_as_uint(f.y);
         }
         if (any_tiny) {
-            // subnormal row factor: 1/r overflows; divide element by element
+            // subnormal row factor: 1/r overflows; scale P and r by 2^64 (exact: |P| <= qmax r)
             const float r = r_io[row];
             if (r > 0.0f && r < FLT_MIN) {
+                const float irs = rcp_refined(r * 0x1p64f);
 #pragma unroll
-                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(__fdiv_rn(T[m][j], r) + MAG);
+                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(fmaf(T[m][j] * 0x1p64f, irs, MAG));
             }
         }
         pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
@@ -320,41 +317,30 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     return true;
 }
 
+// Per-CTA state of the item loop.  The loop runs in three pieces, one per bit width
+// (the heads are visited grouped by width), so each piece is compiled for one width.
 template <int GATE, typename TIn>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
-{
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *stages = smem;
-    Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * a.stage_bytes);
+struct ItemLoop {
+    const DecodeArgs &a;
+    Scratch &sc;
+    uint8_t *stages;
+    TileIdx<4> ix;
+    int tid, lane, count;
+    Cursor cur;
+    long long bh_cur;
+    float beta_cur;
+    bool ok;
+    int slot_next;                      // producer: prefetched slot id of the next item to issue
 
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const long long total = (long long)a.n * a.H;
-    const long long first = blockIdx.x;
-    if (first >= total) return;
-    const int count = int((total - first + gridDim.x - 1) / gridDim.x);
-    constexpr int esz = sizeof(TIn);
-
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sc.full[s], 1);
-            mbar_init(&sc.empty[s], kWarps);
-        }
-        fence_mbarrier_init();
+    __device__ __forceinline__ ItemLoop(const DecodeArgs &a_, Scratch &sc_, uint8_t *stages_, int tid_, int count_)
+        : a(a_), sc(sc_), stages(stages_), ix(tid_), tid(tid_), lane(tid_ & 31), count(count_), ok(true), slot_next(0)
+    {
     }
-    if (tid < 3 * PANEL) sc.invpos[tid / PANEL][tid % PANEL] = kInvPos[tid / PANEL][tid % PANEL];
-    for (int h = tid; h < a.H; h += kThreads) {
-        sc.hoff[h] = a.head_off[h];
-        sc.hord[h] = a.head_order[h];
-        sc.hbits[h] = a.head_bits[h];
-    }
-    __syncthreads();
 
-    const Cursor start = {int(first % a.n), int(first / a.n)};
-
-    // ---- producer (thread 0): bulk-copy item j's inputs into stage j % kStages
-    int slot_next = 0;                  // producer: prefetched slot id of the next item to issue
-    auto issue = [&](int j) {
+    // producer (thread 0): bulk-copy item j's inputs into stage j % kStages
+    __device__ __forceinline__ void issue(int j)
+    {
+        constexpr int esz = sizeof(TIn);
         const int st = j % kStages;
         const int slot = slot_next;
         Cursor pc = {sc.prod_b, sc.prod_h};
@@ -387,89 +373,131 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
                 bulk_g2s(stage + a.blk_cap + 3 * kIoBytes, static_cast<const uint8_t *>(a.alpha) + bh * io, io,
                          &sc.full[st]);
         }
-    };
-    if (tid == 0) {
-        sc.prod_b = start.b;
-        sc.prod_h = start.h;
-        slot_next = __ldg(a.slot_ids + start.b);
-        issue(0);
-        if (count > 1) issue(1);
     }
 
-    const TileIdx<4> ix(tid);
-    const TIn *alpha_g = static_cast<const TIn *>(a.alpha);
-    const TIn *beta_g = static_cast<const TIn *>(a.beta);
+    // Items i .. i_end - 1, all of width BITS (or skipped: bad slot).  Returns false (with
+    // i at the item) when a wait gave up.
+    template <int BITS>
+    __device__ __forceinline__ bool run(int &i, int i_end)
+    {
+        const TIn *alpha_g = static_cast<const TIn *>(a.alpha);
+        const TIn *beta_g = static_cast<const TIn *>(a.beta);
+        for (; i < i_end; ++i) {
+            const int st = i % kStages;
+            if (lane == 0 && i >= 2) {
+                bulk_wait_read<1>();                  // this warp's stores of item i-2 have read their stage
+                mbar_arrive(&sc.empty[(i - 2) % kStages]);
+            }
+            if (tid == 0 && i + 2 < count) {
+                if (i + 2 >= kStages)                // stage (i+2)%4 last held item i-2
+                    ok &= mbar_wait_bounded(&sc.empty[(i + 2) % kStages], uint32_t((i - 2) / kStages) & 1u);
+                issue(i + 2);
+            }
+            // next item: cursor, scalar gates, its stage (waited for before its row table is built)
+            Cursor nxt = cur;
+            nxt.advance(a);
+            const bool has_next = i + 1 < count;
+            const long long bh_next = has_next ? (long long)nxt.b * a.H + sc.hord[nxt.h] : 0;
+            TIn beta_raw = TIn(0), alpha_raw = TIn(0);            // converted when used
+            if (has_next) {
+                beta_raw = beta_g[bh_next];
+                if (GATE == STEPQ_GATE_GDN) alpha_raw = alpha_g[bh_next];
+            }
+            const float4 kqv = *reinterpret_cast<const float4 *>(sc.kqw);
+            const float kq = (kqv.x + kqv.y) + (kqv.z + kqv.w);
+            const int valid = sc.meta[st].valid;
+            if (has_next) ok &= mbar_wait_bounded(&sc.full[(i + 1) % kStages], uint32_t((i + 1) / kStages) & 1u);
+            bool alive;
+            if (!valid) {
+                alive = !__syncthreads_or(!ok);
+                if (alive) {
+                    const StageMeta mn = sc.meta[(i + 1) % kStages];
+                    if (has_next && mn.valid && tid >= DK)
+                        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits,
+                                             to_f32(alpha_raw), sc, tid);
+                    __syncthreads();
+                }
+            } else {
+                alive = decode_item<GATE, TIn, BITS>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
+                                                     alpha_raw, ok);
+            }
+            if (!alive) return false;
+            if (lane == 0) bulk_commit();
+            cur = nxt;
+            bh_cur = bh_next;
+            beta_cur = to_f32(beta_raw);
+        }
+        return true;
+    }
+};
+
+template <int GATE, typename TIn>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *stages = smem;
+    Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * a.stage_bytes);
+
+    const int tid = threadIdx.x;
+    const long long total = (long long)a.n * a.H;
+    const long long first = blockIdx.x;
+    if (first >= total) return;
+    const long long G = gridDim.x;
+    const int count = int((total - first + G - 1) / G);
+    // this CTA's items are first + k G; those with k < end4 are on 4-bit heads, then 6-bit
+    auto class_end = [&](long long e) {
+        return e > first ? int(min((long long)count, (e - first + G - 1) / G)) : 0;
+    };
+    const int end4 = class_end((long long)a.nh4 * a.n);
+    const int end6 = class_end((long long)(a.nh4 + a.nh6) * a.n);
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sc.full[s], 1);
+            mbar_init(&sc.empty[s], kWarps);
+        }
+        fence_mbarrier_init();
+    }
+    if (tid < 3 * PANEL) sc.invpos[tid / PANEL][tid % PANEL] = kInvPos[tid / PANEL][tid % PANEL];
+    for (int h = tid; h < a.H; h += kThreads) {
+        sc.hoff[h] = a.head_off[h];
+        sc.hord[h] = a.head_order[h];
+        sc.hbits[h] = a.head_bits[h];
+    }
+    __syncthreads();
+
+    ItemLoop<GATE, TIn> L(a, sc, stages, tid, count);
+    L.cur = {int(first % a.n), int(first / a.n)};
+    if (tid == 0) {
+        sc.prod_b = L.cur.b;
+        sc.prod_h = L.cur.h;
+        L.slot_next = __ldg(a.slot_ids + L.cur.b);
+        L.issue(0);
+        if (count > 1) L.issue(1);
+    }
 
     // ---- prologue: the first state's row table
-    Cursor cur = start;
-    long long bh_cur = (long long)cur.b * a.H + sc.hord[cur.h];
-    float beta_cur = to_f32(beta_g[bh_cur]);
-    bool ok = mbar_wait_bounded(&sc.full[0], 0u);
+    const TIn *alpha_g = static_cast<const TIn *>(a.alpha);
+    const TIn *beta_g = static_cast<const TIn *>(a.beta);
+    L.bh_cur = (long long)L.cur.b * a.H + sc.hord[L.cur.h];
+    L.beta_cur = to_f32(beta_g[L.bh_cur]);
+    L.ok = mbar_wait_bounded(&sc.full[0], 0u);
     {
         const StageMeta m0 = sc.meta[0];
-        const float al0 = (GATE == STEPQ_GATE_GDN) ? to_f32(alpha_g[bh_cur]) : 1.0f;
+        const float al0 = (GATE == STEPQ_GATE_GDN) ? to_f32(alpha_g[L.bh_cur]) : 1.0f;
         if (m0.valid && tid >= DK) row_table<GATE, TIn>(stages, a, m0.bits, al0, sc, tid);
     }
     __syncthreads();
 
-    int aborted_at = -1;
-    for (int i = 0; i < count; ++i) {
-        const int st = i % kStages;
-        if (lane == 0 && i >= 2) {
-            bulk_wait_read<1>();                      // this warp's stores of item i-2 have read their stage
-            mbar_arrive(&sc.empty[(i - 2) % kStages]);
-        }
-        if (tid == 0 && i + 2 < count) {
-            if (i + 2 >= kStages)                    // stage (i+2)%4 last held item i-2
-                ok &= mbar_wait_bounded(&sc.empty[(i + 2) % kStages], uint32_t((i - 2) / kStages) & 1u);
-            issue(i + 2);
-        }
-        // next item: cursor, scalar gates, its stage (waited for before its row table is built)
-        Cursor nxt = cur;
-        nxt.advance(a);
-        const bool has_next = i + 1 < count;
-        const long long bh_next = has_next ? (long long)nxt.b * a.H + sc.hord[nxt.h] : 0;
-        TIn beta_raw = TIn(0), alpha_raw = TIn(0);            // converted when used
-        if (has_next) {
-            beta_raw = beta_g[bh_next];
-            if (GATE == STEPQ_GATE_GDN) alpha_raw = alpha_g[bh_next];
-        }
-        const float4 kqv = *reinterpret_cast<const float4 *>(sc.kqw);
-        const float kq = (kqv.x + kqv.y) + (kqv.z + kqv.w);
-        const int valid = sc.meta[st].valid, bits = sc.meta[st].bits;
-        if (has_next) ok &= mbar_wait_bounded(&sc.full[(i + 1) % kStages], uint32_t((i + 1) / kStages) & 1u);
-        bool alive;
-        if (!valid) {
-            alive = !__syncthreads_or(!ok);
-            if (alive) {
-                const StageMeta mn = sc.meta[(i + 1) % kStages];
-                if (has_next && mn.valid && tid >= DK)
-                    row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits, to_f32(alpha_raw),
-                                         sc, tid);
-                __syncthreads();
-            }
-        } else if (bits == 4) {
-            alive = decode_item<GATE, TIn, 4>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
-        } else if (bits == 6) {
-            alive = decode_item<GATE, TIn, 6>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
-        } else {
-            alive = decode_item<GATE, TIn, 8>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq, alpha_raw, ok);
-        }
-        if (!alive) {
-            aborted_at = i;
-            break;
-        }
-        if (lane == 0) bulk_commit();
-        cur = nxt;
-        bh_cur = bh_next;
-        beta_cur = to_f32(beta_raw);
-    }
+    int i = 0;
+    const bool done = L.template run<4>(i, end4) && L.template run<6>(i, end6) && L.template run<8>(i, count);
+    const int lane = tid & 31;
     if (lane == 0) bulk_wait_all();
-    if (tid == 0 && aborted_at >= 0) {
+    if (tid == 0 && !done) {
         atomicOr(a.flag, STEPQ_FLAG_TIMEOUT);
         // let the loads still in flight land before the CTA leaves (bounded waits)
-        const int issued = aborted_at + 2 < count ? aborted_at + 3 : count;
-        for (int j = aborted_at; j < issued; ++j)
+        const int issued = i + 2 < count ? i + 3 : count;
+        for (int j = i; j < issued; ++j)
             (void)mbar_wait_bounded(&sc.full[j % kStages], uint32_t(j / kStages) & 1u);
     }
 }
@@ -509,6 +537,15 @@ cudaError_t upload_tables()
     return cudaMemcpyToSymbol(kInvPos, h, sizeof(h));
 }
 
+void count_widths(const uint8_t *bits, int H, DecodeArgs &a)
+{
+    a.nh4 = a.nh6 = 0;
+    for (int h = 0; h < H; ++h) {
+        a.nh4 += bits[h] == 4;
+        a.nh6 += bits[h] == 6;
+    }
+}
+
 }  // namespace
 
 cudaError_t decode_configure(stepq_pool *p)
@@ -539,6 +576,7 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.H = p->H;
     a.Hk = p->Hk;
     a.group = p->H / p->Hk;
+    count_widths(p->bits.data(), p->H, a);
     a.slot_ids = slot_ids;
     a.n = n;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
@@ -710,6 +748,7 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     a.H = H;
     a.Hk = desc->num_key_heads;
     a.group = H / desc->num_key_heads;
+    count_widths(bits, H, a);
     a.slot_ids = slot_ids;
     a.n = n;
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;

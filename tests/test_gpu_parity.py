@@ -166,6 +166,41 @@ def test_power_of_two_fade_equivariance_on_gpu(S):
             assert np.array_equal(A[1] / 2, B[1]) and np.array_equal(A[2] / 2, B[2])
 
 
+def test_decode_extreme_rows_vs_oracle(S):
+    """One step from states with a row of subnormal magnitude whose key component is zero
+    (the refit gives it a subnormal row factor), a state of huge magnitudes, and a zero
+    state: single-step tolerances against the oracle."""
+    rng = np.random.default_rng(11)
+    bits = [4, 6, 8]
+    n, H = 3, 3
+    st = random_states(rng, n, H)
+    st[0, :, 5, :] *= 1e-40                 # subnormal row in every head of request 0
+    st[1] *= 1e30                           # huge magnitudes
+    st[2, 1] = 0                            # zero state
+    ids = np.array([2, 0, 1], np.int32)
+    op = O.OraclePool(3, bits, H)
+    op.load_fp32(ids, st)
+    init = op.slot_bytes(ids)
+    k = np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)])
+    k[0, :, 5] = 0
+    k[0] /= np.linalg.norm(k[0], axis=-1, keepdims=True)
+    x = dict(q=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]), k=k.astype(f32),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.5, 1, (n, H)).astype(f32), beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+    yg, sg, err = _run_gpu(S, bits, H, 0, S.STEPQ_DTYPE_F32, x, init, ids, 3)
+    assert err == 0
+    yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    ob = op.slot_bytes(ids)
+    r0 = np.concatenate([O.split_block(ob[0, o:o + O.block_bytes(b)], b)[1]
+                         for o, b in zip(O.head_offsets(bits)[0], bits)])
+    assert np.any((r0 > 0) & (r0 < np.finfo(np.float32).tiny))      # the subnormal path is reached
+    res = PH.compare_slots(sg, ob, bits)
+    assert res["max_code_diff"] <= 1
+    assert res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
+    assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
+    assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
+
+
 def _run_gpu(S, bits, Hk, gate, dtype, x, init_bytes, ids, num_slots):
     gp = S.Pool(num_slots, bits, Hk, gate, dtype)
     load_bytes(gp, ids, init_bytes)
