@@ -40,7 +40,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=4096)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="mixed6", choices=["mixed6", "uniform4"])
+    ap.add_argument("--variant", default="mixed6", choices=["mixed6", "uniform4", "mixed6p"],
+                    help="mixed6: 6-bit nominal allocation; uniform4; mixed6p: mixed6 plus one FP16 pivot head")
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -134,7 +135,10 @@ class ClockSampler:
 
 
 def block_bytes(bits: int, dk: int = 128, dv: int = 128) -> int:
-    """Packed head block: codes (dk*dv*bits/8 bytes) + fp32 row and column factors."""
+    """Packed head block: codes (dk*dv*bits/8 bytes) + fp32 row and column factors; an FP16
+    pivot head (width 16) is the binary16 state alone."""
+    if bits == 16:
+        return 2 * dk * dv
     return dk * dv * bits // 8 + 4 * dk + 4 * dv
 
 
@@ -186,7 +190,10 @@ def run_reference(args):
     from quantized_gated_delta_b200 import workloads as W
     w = W.make_workload(4, args.variant)
     if w.head_bits is None:
-        bits, _ = O.allocate_bits_dp(list(w.half_life[0]), None, [4, 6, 8], w.avg_bits)
+        if w.n_pivots:
+            bits, _ = O.allocate_bits_pivots(list(w.half_life[0]), None, [4, 6, 8], w.avg_bits, w.n_pivots)
+        else:
+            bits, _ = O.allocate_bits_dp(list(w.half_life[0]), None, [4, 6, 8], w.avg_bits)
     else:
         bits = list(w.head_bits[0])
     pool, sl, xs = _oracle_sample(w, bits, 16)
@@ -232,7 +239,12 @@ def main():
 
     w = W.make_workload(4, args.variant)
     w.seed = D.shard_seed(w.seed, rank)              # each rank serves its own requests
-    bits = w.head_bits[0] if w.head_bits is not None else stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
+    if w.head_bits is not None:
+        bits = w.head_bits[0]
+    elif w.n_pivots:
+        bits = stepq.stepq_allocate_bits_pivots(w.half_life[0], None, (4, 6, 8), w.avg_bits, w.n_pivots)
+    else:
+        bits = stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
     bits = np.asarray(bits, dtype=np.uint8)
     pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
     slots = torch.from_numpy(w.slot_ids).cuda()
@@ -341,7 +353,7 @@ def main():
                          "kernel": "decode_kernel", "avg_kernel_us": avg_kernel_s * 1e6},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * (2 if int(np.sum(bits == 16)) else 1),   # + pivot kernel
             "clocks": clocks,
             "cpu_baseline": base,
         }

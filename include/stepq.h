@@ -36,6 +36,10 @@
  *     8-bit: one per byte); the element order in the stream is panel-major: 16-column
  *     panels, each panel row-major, i.e. stream index = (j / 16) * d_k * 16 + i * 16 + j % 16
  *   - a zero-filled block (r = c = 0) is the zero state
+ *   - FP16 pivot heads (width 16; STEPQuant summary, "Method" para 2: the highest-risk
+ *     units are kept in FP16 as sparse pivots): the block is the state itself, d_k x d_v
+ *     IEEE binary16 values, row-major, little-endian (32768 bytes), no scales; each step
+ *     stores the updated state rounded to binary16 (nearest, ties to even)
  */
 #ifndef STEPQ_H
 #define STEPQ_H
@@ -61,7 +65,7 @@ typedef enum {
     STEPQ_INVALID_ARG = -1,              /* null pointer, bad size or alignment, bad count   */
     STEPQ_OUT_OF_MEMORY = -2,            /* device or host allocation failed                 */
     STEPQ_CUDA_ERROR = -3,               /* a CUDA runtime call or kernel launch failed      */
-    STEPQ_UNSUPPORTED = -4,              /* d_k or d_v != 128, or a bit width not in {4,6,8} */
+    STEPQ_UNSUPPORTED = -4,              /* d_k or d_v != 128, or a width not in {4,6,8,16}  */
     STEPQ_DEVICE_FLAG = -5               /* the pool's sticky device flag was set            */
 } stepq_status;
 
@@ -85,8 +89,9 @@ typedef struct {
                                             STEPQ_GATE_KDA: alpha [n, H, d_k]                 */
     int32_t in_dtype;                    /* STEPQ_DTYPE_F32 or _BF16: dtype of q, k, v,
                                             alpha and beta (y is always float32)             */
-    const uint8_t *head_bits;            /* HOST array [H], each 4, 6 or 8 (from an offline
-                                            allocation, e.g. stepq_allocate_bits)            */
+    const uint8_t *head_bits;            /* HOST array [H], each 4, 6, 8 or 16 (16: an FP16
+                                            pivot head; from an offline allocation, e.g.
+                                            stepq_allocate_bits_pivots)                      */
 } stepq_pool_desc;
 
 /* Create a pool and zero it (every slot holds the zero state).  The descriptor and
@@ -177,6 +182,15 @@ STEPQ_API int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out);
  * distinct widths in {4, 6, 8}.  Returns STEPQ_INVALID_ARG when no assignment fits. */
 STEPQ_API int stepq_allocate_bits(const double *half_life, const double *distortion, int32_t N,
                         const uint8_t *cand, int32_t C, double avg_bits, uint8_t *bits_out);
+
+/* Lifetime-aware allocation with FP16 pivots (host, offline).  [SUM Method, para 2]
+ * The n_pivots units of highest risk w_u * D_u(b_max) (b_max the widest candidate; ties go
+ * to the lower index) get width 16 and sit outside the budget; the other N - n_pivots units
+ * are allocated as by stepq_allocate_bits with the budget floor((N - n_pivots) * avg_bits).
+ * Returns STEPQ_INVALID_ARG also for n_pivots outside [0, N]. */
+STEPQ_API int stepq_allocate_bits_pivots(const double *half_life, const double *distortion, int32_t N,
+                                         const uint8_t *cand, int32_t C, double avg_bits, int32_t n_pivots,
+                                         uint8_t *bits_out);
 
 /* Static description of a status code. */
 STEPQ_API const char *stepq_status_string(int status);

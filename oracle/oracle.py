@@ -65,6 +65,8 @@ def _load():
         "oracle_pool_load": (L, [I, I, I, P, I, P, P, I, P, I]),
         "oracle_pool_dump": (I, [I, I, I, P, I, P, P, I, P, I]),
         "oracle_fp_decode_step": (None, [I, I, I, I, I, I, P, P, P, P, P, P, P, I, I]),
+        "oracle_fp16_encode": (None, [L, P, P]),
+        "oracle_fp16_decode": (None, [L, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -131,6 +133,26 @@ def split_block(blk: np.ndarray, bits: int, dk: int = 128, dv: int = 128):
     r = blk[cb:cb + 4 * dk].view(np.float32).copy()
     c = blk[cb + 4 * dk:cb + 4 * dk + 4 * dv].view(np.float32).copy()
     return Q, r, c
+
+
+def fp16_encode(x) -> np.ndarray:
+    """Nearest binary16 values of x (float64 array, ties to even), as uint16 bit patterns."""
+    x = _c(x, np.float64)
+    out = np.zeros(x.shape, dtype=np.uint16)
+    _load().oracle_fp16_encode(x.size, _p(x), _p(out))
+    return out
+
+
+def fp16_decode(h) -> np.ndarray:
+    h = _c(h, np.uint16)
+    out = np.zeros(h.shape, dtype=np.float64)
+    _load().oracle_fp16_decode(h.size, _p(h), _p(out))
+    return out
+
+
+def pivot_state(blk: np.ndarray, dk: int = 128, dv: int = 128) -> np.ndarray:
+    """FP16 pivot head block bytes -> the state's binary16 bit patterns [dk, dv]."""
+    return _c(blk, np.uint8)[:2 * dk * dv].view(np.uint16).reshape(dk, dv).copy()
 
 
 def make_block(Q, r, c, bits: int) -> np.ndarray:
@@ -203,7 +225,8 @@ def step_state(Q, r, c, bits: int, q, k, v, alpha, beta: float):
 
 class OraclePool:
     """Host pool with the packed layout: slot-major, heads in order, each head block
-    = [codes | r fp32[dk] | c fp32[dv]].  A zeroed pool is the zero state."""
+    = [codes | r fp32[dk] | c fp32[dv]] (an FP16 pivot head, width 16: the state as
+    binary16 values).  A zeroed pool is the zero state."""
 
     def __init__(self, num_slots: int, head_bits, num_key_heads: int, gate_mode: int = 0,
                  dk: int = 128, dv: int = 128):
@@ -223,6 +246,9 @@ class OraclePool:
         return self.data[o:o + block_bytes(int(self.head_bits[h]), self.dk, self.dv)]
 
     def state(self, slot: int, h: int):
+        """(Q, r, c) of a quantized head; the binary16 bit patterns of an FP16 pivot head."""
+        if int(self.head_bits[h]) == 16:
+            return pivot_state(self.block(slot, h), self.dk, self.dv)
         return split_block(self.block(slot, h), int(self.head_bits[h]), self.dk, self.dv)
 
     def set_state(self, slot: int, h: int, Q, r, c):
@@ -327,6 +353,29 @@ def allocate_bits_bruteforce(half_life, distortion, cand, avg_bits):
         if best is None or obj < best:
             best, best_bits = obj, [cand[c] for c in combo]
     return best_bits, best
+
+
+def select_pivots(half_life, distortion, cand, n_pivots: int):
+    """Indices of the FP16 pivot units ([SUM] Method para 2: the highest-risk units are kept
+    in FP16).  Reading: risk = lifetime weight x the distortion left at the widest candidate
+    width; the n_pivots units of highest risk, ties to the lower index."""
+    cand = list(cand)
+    top = cand.index(max(cand))
+    risk = [(-lifetime_weight(h) * _distortion(distortion, u, top, cand), u) for u, h in enumerate(half_life)]
+    return sorted(u for _, u in sorted(risk)[:n_pivots])
+
+
+def allocate_bits_pivots(half_life, distortion, cand, avg_bits, n_pivots: int):
+    """Pivots first (width 16, outside the budget), then the exact DP over the other units
+    with the budget floor((N - n_pivots) * avg_bits)."""
+    piv = set(select_pivots(half_life, distortion, cand, n_pivots))
+    rest = [u for u in range(len(half_life)) if u not in piv]
+    sub_d = None if distortion is None else [distortion[u] for u in rest]
+    bits_rest, obj = allocate_bits_dp([half_life[u] for u in rest], sub_d, cand, avg_bits)
+    bits = [16] * len(half_life)
+    for u, b in zip(rest, bits_rest):
+        bits[u] = b
+    return bits, obj
 
 
 def allocate_bits_dp(half_life, distortion, cand, avg_bits):

@@ -47,7 +47,77 @@ long oracle_codes_bytes(int bits, int dk, int dv) { return (long)dk * dv * bits 
 
 long oracle_block_bytes(int bits, int dk, int dv)
 {
+    if (bits == 16) return 2L * dk * dv;               /* FP16 pivot head: the state, no scales */
     return oracle_codes_bytes(bits, dk, dv) + 4L * dk + 4L * dv;
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP16 pivot heads ([SUM] Method para 2: the highest-risk units are kept in   */
+/* FP16 as sparse pivots)                                                      */
+/* ------------------------------------------------------------------------- */
+/* A head of width 16 stores its state as IEEE binary16 values, row-major, element (i, j)
+ * at byte 2 (i d_v + j), little-endian, with no scales.  Reading: the step fades, writes
+ * and reads out as for every head; the updated state is rounded to fp32 (the fp32 store
+ * that precedes the fit of a quantized head) and then to binary16, nearest, ties to even. */
+
+/* Nearest binary16 value of x (ties to even), as its bit pattern.  binary16: 1 sign bit,
+ * 5 exponent bits (bias 15), 10 fraction bits; subnormals are multiples of 2^-24; the
+ * largest finite value is 65504 and everything from 65520 (the halfway point to 2^16) up
+ * rounds to infinity. */
+uint16_t oracle_fp16_from_double(double x)
+{
+    if (isnan(x)) return 0x7E00;
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    const double a = fabs(x);
+    if (a >= 65520.0) return sign | 0x7C00;
+    if (a < 0x1p-14) {
+        /* subnormal range: an integer multiple of 2^-24 (1024 of them is the smallest normal) */
+        return sign | (uint16_t)nearbyint(a * 0x1p24);
+    }
+    int e;
+    frexp(a, &e);
+    e -= 1;                                           /* a in [2^e, 2^(e+1)), -14 <= e <= 15 */
+    double m = nearbyint(ldexp(a, 10 - e));           /* 1024 .. 2048: 11 significant bits */
+    if (m == 2048.0) {
+        m = 1024.0;
+        e += 1;
+    }
+    return sign | (uint16_t)((e + 15) << 10) | (uint16_t)(m - 1024.0);
+}
+
+double oracle_fp16_to_double(uint16_t h)
+{
+    const int e = (h >> 10) & 31, f = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)f, -24);
+    else if (e == 31) v = f ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + f), e - 25);
+    return (h & 0x8000) ? -v : v;
+}
+
+void oracle_fp16_encode(long n, const double *x, uint16_t *out)
+{
+    for (long e = 0; e < n; e++) out[e] = oracle_fp16_from_double(x[e]);
+}
+
+void oracle_fp16_decode(long n, const uint16_t *in, double *out)
+{
+    for (long e = 0; e < n; e++) out[e] = oracle_fp16_to_double(in[e]);
+}
+
+static void read_pivot(const uint8_t *blk, long ne, double *S)
+{
+    for (long e = 0; e < ne; e++)
+        S[e] = oracle_fp16_to_double((uint16_t)(blk[2 * e] | (blk[2 * e + 1] << 8)));
+}
+
+static void write_pivot(uint8_t *blk, long ne, const double *S)
+{
+    for (long e = 0; e < ne; e++) {
+        const uint16_t h = oracle_fp16_from_double((double)(float)S[e]);
+        blk[2 * e] = (uint8_t)(h & 0xFF);
+        blk[2 * e + 1] = (uint8_t)(h >> 8);
+    }
 }
 
 /* Position of element (i, j) in the code stream: panel-major, row-major inside a panel. */
@@ -258,6 +328,21 @@ long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int3
         int bits = head_bits[h];
         int g = h / group;
         long ne = (long)dk * dv;
+        if (bits == 16) {
+            double *S = (double *)malloc((size_t)ne * sizeof(double));
+            double *yd = (double *)malloc((size_t)dv * sizeof(double));
+            float *alp = (float *)malloc(4L * dk);
+            uint8_t *pblk = pool + (long)slot * stride + offsets[h];
+            for (int i = 0; i < dk; i++)
+                alp[i] = gate_mode == 0 ? alpha[(long)b * H + h] : alpha[((long)b * H + h) * dk + i];
+            read_pivot(pblk, ne, S);
+            oracle_delta_step(dk, dv, S, q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
+                              v + ((long)b * H + h) * dv, alp, beta[(long)b * H + h], yd);
+            for (int j = 0; j < dv; j++) y[((long)b * H + h) * dv + j] = (float)yd[j];
+            write_pivot(pblk, ne, S);
+            free(S); free(yd); free(alp);
+            continue;
+        }
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         int32_t *Q2 = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
@@ -293,6 +378,13 @@ long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_s
         int slot = slot_ids[b];
         if (slot < 0 || slot >= num_slots) { bad |= 1; continue; }
         long ne = (long)dk * dv;
+        if (head_bits[h] == 16) {
+            double *Sd = (double *)malloc((size_t)ne * sizeof(double));
+            for (long e = 0; e < ne; e++) Sd[e] = (double)S[it * ne + e];
+            write_pivot(pool + (long)slot * stride + offsets[h], ne, Sd);
+            free(Sd);
+            continue;
+        }
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
         clipped += oracle_quantize(head_bits[h], dk, dv, S + it * ne, Q, r, c);
@@ -317,6 +409,13 @@ int oracle_pool_dump(int H, int dk, int dv, const int32_t *head_bits, int num_sl
         int slot = slot_ids[b];
         if (slot < 0 || slot >= num_slots) { bad |= 1; continue; }
         long ne = (long)dk * dv;
+        if (head_bits[h] == 16) {
+            double *Sp = (double *)malloc((size_t)ne * sizeof(double));
+            read_pivot(pool + (long)slot * stride + offsets[h], ne, Sp);
+            for (long e = 0; e < ne; e++) S[it * ne + e] = (float)Sp[e];
+            free(Sp);
+            continue;
+        }
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
         double *Sd = (double *)malloc((size_t)ne * sizeof(double));

@@ -61,7 +61,7 @@ const char *stepq_status_string(int status)
     case STEPQ_INVALID_ARG: return "invalid argument";
     case STEPQ_OUT_OF_MEMORY: return "out of memory";
     case STEPQ_CUDA_ERROR: return "CUDA error";
-    case STEPQ_UNSUPPORTED: return "unsupported configuration (d_k = d_v = 128, bits in {4, 6, 8})";
+    case STEPQ_UNSUPPORTED: return "unsupported configuration (d_k = d_v = 128, bits in {4, 6, 8, 16})";
     case STEPQ_DEVICE_FLAG: return "device flag set (bad slot id or kernel wait timeout)";
     default: return "unknown status";
     }
@@ -79,7 +79,7 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     if (desc->d_k != stepq::DK || desc->d_v != stepq::DV) return STEPQ_UNSUPPORTED;
     for (int h = 0; h < desc->num_heads; ++h) {
         const int b = desc->head_bits[h];
-        if (b != 4 && b != 6 && b != 8) return STEPQ_UNSUPPORTED;
+        if (b != 4 && b != 6 && b != 8 && b != 16) return STEPQ_UNSUPPORTED;
     }
     stepq_pool *p = new (std::nothrow) stepq_pool();
     if (!p) return STEPQ_OUT_OF_MEMORY;
@@ -94,7 +94,10 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     for (int h = 0; h < p->H; ++h) {
         p->offs[h] = off;
         off += block_bytes(p->bits[h]);
-        if (block_bytes(p->bits[h]) > p->max_block) p->max_block = block_bytes(p->bits[h]);
+        if (p->bits[h] == 16)
+            ++p->npiv;
+        else if (block_bytes(p->bits[h]) > p->max_block)
+            p->max_block = block_bytes(p->bits[h]);
     }
     p->slot_stride = off;
     p->total = off * (long long)p->num_slots;
@@ -110,9 +113,10 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     if (e == cudaSuccess) e = cudaMemcpy(p->d_offs, p->offs.data(), sizeof(long long) * p->H, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_bits, p->bits.data(), size_t(p->H), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) {
-        // the decode kernel visits heads grouped by bit width (stable within a width)
+        // the decode kernel visits heads grouped by bit width (stable within a width); the
+        // FP16 pivot heads come last and go to their own kernel
         std::vector<int32_t> order;
-        for (int w = 4; w <= 8; w += 2)
+        for (int w : {4, 6, 8, 16})
             for (int h = 0; h < p->H; ++h)
                 if (p->bits[h] == w) order.push_back(h);
         e = cudaMemcpy(p->d_order, order.data(), sizeof(int32_t) * p->H, cudaMemcpyHostToDevice);

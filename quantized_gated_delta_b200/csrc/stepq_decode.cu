@@ -33,6 +33,7 @@
 // from the stage (warp 0 also r).  Each state is read from HBM once and written once.
 #include <cfloat>
 #include <cstdint>
+#include <cuda_fp16.h>
 
 #include "stepq_internal.h"
 #include "stepq_tile.cuh"
@@ -63,6 +64,7 @@ struct DecodeArgs {
     const int32_t *head_order;      // processing order of the heads (grouped by bit width)
     int num_slots, H, Hk, group;
     int nh4, nh6;                   // heads of width 4 and 6 (visited first, in that order)
+    int Hq;                         // quantized heads: the first Hq entries of head_order
     const int32_t *slot_ids;
     int n;
     int step_b, step_h;             // gridDim.x in head-major items = step_h * n + step_b
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * a.stage_bytes);
 
     const int tid = threadIdx.x;
-    const long long total = (long long)a.n * a.H;
+    const long long total = (long long)a.n * a.Hq;
     const long long first = blockIdx.x;
     if (first >= total) return;
     const long long G = gridDim.x;
@@ -499,6 +501,120 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
         const int issued = i + 2 < count ? i + 3 : count;
         for (int j = i; j < issued; ++j)
             (void)mbar_wait_bounded(&sc.full[j % kStages], uint32_t(j / kStages) & 1u);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// FP16 pivot heads (STEPQuant summary, "Method" para 2: the highest-risk units are kept in
+// FP16).  The state is binary16, row-major; the step fades, writes and reads out as for the
+// quantized heads and stores the updated state rounded to binary16 (nearest, ties to even),
+// with no fit.  One CTA of 256 threads per (request, pivot head): warp w owns the 16-column
+// panel w, lane l rows l + 32 m, the same column dot products as the quantized kernel with
+// rho_i = alpha_i and no column factor.
+// ------------------------------------------------------------------------------------------
+template <int GATE, typename TIn>
+__global__ void __launch_bounds__(kThreads) pivot_kernel(const DecodeArgs a, int npiv)
+{
+    __shared__ float4 wlo[DK], whi[DK], wrk[DK];
+    __shared__ float xd[DV];
+    __shared__ float kqw[4];
+    const int tid = threadIdx.x;
+    const long long item = blockIdx.x;
+    const int b = int(item / npiv);
+    const int h = a.head_order[a.Hq + int(item % npiv)];
+    const int slot = a.slot_ids[b];
+    if (slot < 0 || slot >= a.num_slots) {
+        if (tid == 0) atomicOr(a.flag, STEPQ_FLAG_BAD_SLOT);
+        return;
+    }
+    const int g = h / a.group;
+    const long long bh = (long long)b * a.H + h;
+    const long long kqrow = (long long)b * a.Hk + g;
+    uint16_t *blk = reinterpret_cast<uint16_t *>(a.pool + (long long)slot * a.slot_stride + a.head_off[h]);
+    const TIn *qg = static_cast<const TIn *>(a.q) + kqrow * DK;
+    const TIn *kg = static_cast<const TIn *>(a.k) + kqrow * DK;
+    const TIn *vg = static_cast<const TIn *>(a.v) + bh * DV;
+    const TIn *ag = static_cast<const TIn *>(a.alpha);
+    const float beta = to_f32(static_cast<const TIn *>(a.beta)[bh]);
+
+    // row tables (threads 0..127, row tid) and k.q
+    if (tid < DK) {
+        const float al = to_f32(GATE == STEPQ_GATE_KDA ? ag[bh * DK + tid] : ag[bh]);
+        const float k = to_f32(kg[tid]), q = to_f32(qg[tid]);
+        const float rk = al * k, rq = al * q;
+        wlo[tid] = make_float4(rk, rk, rq, rq);
+        whi[tid] = make_float4(rq, rq, rk, rk);
+        wrk[tid] = make_float4(al, al, k, k);
+        float kq = k * q;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) kq += __shfl_xor_sync(kFull, kq, o);
+        if ((tid & 31) == 0) kqw[tid >> 5] = kq;
+    }
+    const TileIdx<4> ix(tid);
+    const int lane = ix.lane, panel = ix.panel;
+    const bool upper = (lane & 16) != 0;
+    const int col = lane & 15;
+    float T[4][PANEL];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(blk + ix.row(m) * DV + panel * PANEL);
+        const uint4 lo = src[0], hi = src[1];
+        const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wv[e]));
+            T[m][2 * e] = f.x;
+            T[m][2 * e + 1] = f.y;
+        }
+    }
+    __syncthreads();
+    const float kq = (kqw[0] + kqw[1]) + (kqw[2] + kqw[3]);
+
+    // u_j (lanes 0..15) and y'_j (lanes 16..31) of the panel's columns
+    const float4 *wt = upper ? whi : wlo;
+    float4 w[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) w[m] = wt[ix.row(m)];
+    float A[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 2) {
+        float2 s1 = fmul2(make_float2(T[0][j], T[0][j + 1]), make_float2(w[0].x, w[0].y));
+        float2 s2 = fmul2(make_float2(T[0][j], T[0][j + 1]), make_float2(w[0].z, w[0].w));
+#pragma unroll
+        for (int m = 1; m < 4; ++m) {
+            s1 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].x, w[m].y), s1);
+            s2 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].z, w[m].w), s2);
+        }
+        A[j] = s1.x + __shfl_xor_sync(kFull, s2.x, 16);
+        A[j + 1] = s1.y + __shfl_xor_sync(kFull, s2.y, 16);
+    }
+    reduce_scatter<PANEL, 4, 8, false>(A, lane);
+    const float delta = beta * (to_f32(vg[panel * PANEL + col]) - A[0]);
+    const float dpair = __shfl_xor_sync(kFull, delta, 16);
+    st_global_if(upper, a.y + bh * DV + panel * PANEL + col, fmaf(dpair, kq, A[0]));
+    st_shared_if(!upper, xd + panel * PANEL + col, delta);
+    __syncwarp();
+    float dd[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(xd + panel * PANEL + j);
+        dd[j] = t4.x; dd[j + 1] = t4.y; dd[j + 2] = t4.z; dd[j + 3] = t4.w;
+    }
+    // S_ij = alpha_i S_ij + k_i d_j, stored as binary16 in place
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float4 rk = wrk[ix.row(m)];
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            float2 t2 = fmul2(make_float2(T[m][j], T[m][j + 1]), make_float2(rk.x, rk.y));
+            t2 = ffma2(make_float2(rk.z, rk.w), make_float2(dd[j], dd[j + 1]), t2);
+            const __half2 hv = __float22half2_rn(t2);
+            o[j / 2] = *reinterpret_cast<const uint32_t *>(&hv);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(blk + ix.row(m) * DV + panel * PANEL);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
 }
 
@@ -584,22 +700,41 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.flag = p->d_flag;
     a.blk_cap = p->blk_cap;
     a.stage_bytes = p->stage_bytes;
+    a.Hq = p->H - p->npiv;
     // items are dealt round-robin in head-major order, so the CTAs resident at any moment
     // work on one or two heads (one bit width: one code path in the instruction caches)
-    const long long total = (long long)n * p->H;
-    const int grid = int(total < p->decode_grid ? total : p->decode_grid);
-    a.step_b = grid % n;
-    a.step_h = grid / n;
-    if (p->gate_mode == STEPQ_GATE_GDN) {
-        if (p->in_dtype == STEPQ_DTYPE_BF16)
-            decode_kernel<STEPQ_GATE_GDN, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
-        else
-            decode_kernel<STEPQ_GATE_GDN, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
-    } else {
-        if (p->in_dtype == STEPQ_DTYPE_BF16)
-            decode_kernel<STEPQ_GATE_KDA, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
-        else
-            decode_kernel<STEPQ_GATE_KDA, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+    const long long total = (long long)n * a.Hq;
+    if (total > 0) {
+        const int grid = int(total < p->decode_grid ? total : p->decode_grid);
+        a.step_b = grid % n;
+        a.step_h = grid / n;
+        if (p->gate_mode == STEPQ_GATE_GDN) {
+            if (p->in_dtype == STEPQ_DTYPE_BF16)
+                decode_kernel<STEPQ_GATE_GDN, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+            else
+                decode_kernel<STEPQ_GATE_GDN, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+        } else {
+            if (p->in_dtype == STEPQ_DTYPE_BF16)
+                decode_kernel<STEPQ_GATE_KDA, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+            else
+                decode_kernel<STEPQ_GATE_KDA, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (p->npiv > 0) {
+        const unsigned pgrid = unsigned(n) * unsigned(p->npiv);
+        if (p->gate_mode == STEPQ_GATE_GDN) {
+            if (p->in_dtype == STEPQ_DTYPE_BF16)
+                pivot_kernel<STEPQ_GATE_GDN, uint16_t><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+            else
+                pivot_kernel<STEPQ_GATE_GDN, float><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+        } else {
+            if (p->in_dtype == STEPQ_DTYPE_BF16)
+                pivot_kernel<STEPQ_GATE_KDA, uint16_t><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+            else
+                pivot_kernel<STEPQ_GATE_KDA, float><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+        }
     }
     return cudaGetLastError();
 }
@@ -748,6 +883,7 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     a.H = H;
     a.Hk = desc->num_key_heads;
     a.group = H / desc->num_key_heads;
+    a.Hq = H;
     count_widths(bits, H, a);
     a.slot_ids = slot_ids;
     a.n = n;

@@ -13,13 +13,14 @@ struct stepq_pool {
     std::vector<long long> offs;        // [H] byte offset of each head block in a slot
     long long slot_stride = 0;          // bytes per slot
     long long total = 0;                // bytes of the pool
-    int max_block = 0;                  // largest head block (bytes)
+    int max_block = 0;                  // largest quantized head block (bytes)
+    int npiv = 0;                       // FP16 pivot heads (width 16), visited after the others
     int device = 0;
     int num_sms = 0;
     uint8_t *d_pool = nullptr;          // [num_slots * slot_stride]
     long long *d_offs = nullptr;        // [H]
     uint8_t *d_bits = nullptr;          // [H]
-    int32_t *d_order = nullptr;         // [H] head processing order (grouped by bit width)
+    int32_t *d_order = nullptr;         // [H] head processing order (widths 4, 6, 8, then pivots)
     int *d_flag = nullptr;              // sticky device flag (STEPQ_FLAG_* bits)
     int decode_grid = 0;                // persistent CTAs for the decode kernel
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel

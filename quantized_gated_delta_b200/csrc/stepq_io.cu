@@ -1,9 +1,11 @@
 // stepq_io.cu -- pool I/O kernels of libstepq (sm_100a): quantize fp32 states into the
 // pool (clip-free dual-axis fit + round-half-even, STEPQuant summary "Method"), dequantize
-// them back, and copy packed slot images in and out.  One CTA of 256 threads per
-// (request, head) state, each thread a 4-row x 16-column register tile.
+// them back (FP16 pivot heads: round to binary16 and back), and copy packed slot images in
+// and out.  One CTA of 256 threads per (request, head) state, each thread a 4-row x
+// 16-column register tile.
 #include <cfloat>
 #include <cstdint>
+#include <cuda_fp16.h>
 
 #include "stepq_internal.h"
 #include "stepq_tile.cuh"
@@ -156,7 +158,12 @@ __global__ void __launch_bounds__(256) load_fp32_kernel(const IoArgs a, const fl
     switch (a.head_bits[h]) {
     case 4: load_fp32_item<4>(a, blk, Si, ix, rp, xc); break;
     case 6: load_fp32_item<6>(a, blk, Si, ix, rp, xc); break;
-    default: load_fp32_item<8>(a, blk, Si, ix, rp, xc); break;
+    case 8: load_fp32_item<8>(a, blk, Si, ix, rp, xc); break;
+    default: {
+        // FP16 pivot head: the state rounded to binary16 (nearest, ties to even)
+        __half *dst = reinterpret_cast<__half *>(blk);
+        for (int e = threadIdx.x; e < DK * DV; e += blockDim.x) dst[e] = __float2half_rn(Si[e]);
+    }
     }
 }
 
@@ -201,7 +208,11 @@ __global__ void __launch_bounds__(256) dump_fp32_kernel(const IoArgs a, float *S
     switch (a.head_bits[h]) {
     case 4: dump_fp32_item<4>(blk, Si, ix); break;
     case 6: dump_fp32_item<6>(blk, Si, ix); break;
-    default: dump_fp32_item<8>(blk, Si, ix); break;
+    case 8: dump_fp32_item<8>(blk, Si, ix); break;
+    default: {
+        const __half *src = reinterpret_cast<const __half *>(blk);
+        for (int e = threadIdx.x; e < DK * DV; e += blockDim.x) Si[e] = __half2float(src[e]);
+    }
     }
 }
 

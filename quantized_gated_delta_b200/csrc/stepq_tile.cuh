@@ -20,7 +20,11 @@ constexpr int NPANEL = DV / PANEL;
 
 __host__ __device__ constexpr int qmax_of(int bits) { return (1 << (bits - 1)) - 1; }
 __host__ __device__ constexpr int codes_bytes(int bits) { return DK * DV * bits / 8; }
-__host__ __device__ constexpr int block_bytes(int bits) { return codes_bytes(bits) + 4 * DK + 4 * DV; }
+// head block: codes + r + c; an FP16 pivot head (width 16) holds the state as binary16 values
+__host__ __device__ constexpr int block_bytes(int bits)
+{
+    return bits == 16 ? 2 * DK * DV : codes_bytes(bits) + 4 * DK + 4 * DV;
+}
 // bytes of one row's 16 codes inside a panel, and the panel size
 __host__ __device__ constexpr int seg_bytes(int bits) { return PANEL * bits / 8; }
 __host__ __device__ constexpr int panel_bytes(int bits) { return DK * seg_bytes(bits); }

@@ -28,6 +28,7 @@ EXPORTED = [
     "stepq_pool_load_fp32", "stepq_pool_load_packed", "stepq_pool_dump_fp32",
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
+    "stepq_allocate_bits_pivots",
 ]
 
 
@@ -67,6 +68,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_decode_step": [P, P, I, P, P, P, P, P, P, P],
         "stepq_pool_get_error": [P, ctypes.POINTER(I)],
         "stepq_allocate_bits": [P, P, I, P, I, ctypes.c_double, P],
+        "stepq_allocate_bits_pivots": [P, P, I, P, I, ctypes.c_double, I, P],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
@@ -191,6 +193,20 @@ def stepq_allocate_bits(half_life, distortion=None, cand=(4, 6, 8), avg_bits: fl
     _check(load_library().stepq_allocate_bits(hl.ctypes.data, None if dist is None else dist.ctypes.data,
                                               len(hl), cd.ctypes.data, len(cd), float(avg_bits),
                                               out.ctypes.data), "stepq_allocate_bits")
+    return out
+
+
+def stepq_allocate_bits_pivots(half_life, distortion=None, cand=(4, 6, 8), avg_bits: float = 6.0,
+                               n_pivots: int = 0) -> np.ndarray:
+    hl = np.ascontiguousarray(half_life, dtype=np.float64)
+    cd = np.ascontiguousarray(cand, dtype=np.uint8)
+    dist = None if distortion is None else np.ascontiguousarray(distortion, dtype=np.float64)
+    if dist is not None and dist.shape != (len(hl), len(cd)):
+        raise ValueError("distortion must be [N, C]")
+    out = np.zeros(len(hl), dtype=np.uint8)
+    _check(load_library().stepq_allocate_bits_pivots(hl.ctypes.data, None if dist is None else dist.ctypes.data,
+                                                     len(hl), cd.ctypes.data, len(cd), float(avg_bits),
+                                                     int(n_pivots), out.ctypes.data), "stepq_allocate_bits_pivots")
     return out
 
 

@@ -70,6 +70,7 @@ class Workload:
     slot_ids: np.ndarray      # [B] int32, distinct, in [0, num_slots)
     head_bits: np.ndarray | None = None   # [layers, H] fixed widths, or None (set by an allocator)
     avg_bits: float = 6.0     # nominal average width for the allocator
+    n_pivots: int = 0         # FP16 pivot heads per layer chosen by the allocator
     layers: int = 1
     warmup_steps: int = 32
     kda_mu: np.ndarray | None = None      # [layers, H]
@@ -121,8 +122,21 @@ def make_workload(config: int, variant: str = "mixed6", batch: int | None = None
     3  KDA layer: B=256, H=Hk=32, T=64, bf16, per-channel gates, 6-bit nominal
     4  high-concurrency GDN pool: B=512 of 1024 slots (random slot ids), H=32, Hk=16, T=256,
        bf16; variant "mixed6" (6-bit nominal) or "uniform4"
+    Variant "mixed6p" (configs 2-4): 6-bit nominal plus one FP16 pivot head per layer, the
+    smallest nonzero share at 32 heads (the pages keep 1.39% of the heads in FP16)
     5  36-layer GDN stack: H=32, Hk=16, T=32 per layer, B in {64, 256, 1024} (``batch``), bf16
     """
+    if variant not in ("mixed6", "mixed6p", "uniform4") or (variant == "uniform4" and config != 4) \
+            or (variant == "mixed6p" and config not in (2, 3, 4)):
+        raise ValueError("variant %r of workload %r" % (variant, config))
+    w = _make_workload(config, variant, batch)
+    if variant == "mixed6p":
+        w.n_pivots = 1
+        w.name += "_p"
+    return w
+
+
+def _make_workload(config: int, variant: str, batch: int | None) -> Workload:
     if config == 1:
         return Workload("gdn_toy", B=4, H=4, Hk=4, T=16, gate_mode=GATE_GDN, in_dtype=DTYPE_FP32,
                         num_slots=4, seed=0,
@@ -142,13 +156,11 @@ def make_workload(config: int, variant: str = "mixed6", batch: int | None = None
                         slot_ids=np.arange(256, dtype=np.int32))
     if config == 4:
         perm = _rng(4, 2000).permutation(1024).astype(np.int32)
-        w = Workload("gdn_pool_" + variant, B=512, H=32, Hk=16, T=256, gate_mode=GATE_GDN,
+        w = Workload("gdn_pool_" + variant.rstrip("p"), B=512, H=32, Hk=16, T=256, gate_mode=GATE_GDN,
                      in_dtype=DTYPE_BF16, num_slots=1024, seed=4,
                      half_life=_loguniform_half_life(4, 1, 32), slot_ids=perm[:512])
         if variant == "uniform4":
             w.head_bits = np.full((1, 32), 4, dtype=np.int32)
-        elif variant != "mixed6":
-            raise ValueError(variant)
         return w
     if config == 5:
         B = 1024 if batch is None else int(batch)

@@ -13,12 +13,17 @@ R_ULP = 8                   # row factors r within 8 ulp of the oracle's
 C_ULP = 4                   # column factors c within 4 ulp
 Y_MAX_REL = 1e-4            # per (request, head): max_j |dy_j| / max_j |y_j|
 Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
+PIVOT_ULP = 1               # FP16 pivot states: binary16 values within 1 ulp ...
+PIVOT_FLIP_RATE = 1e-3      # ... and off by one ulp at most at this rate
 
 
 def head_bits(w: W.Workload, layer: int = 0) -> np.ndarray:
     """Fixed widths of the workload, else the oracle's lifetime-aware allocation."""
     if w.head_bits is not None:
         return np.asarray(w.head_bits[layer], dtype=np.int32)
+    if w.n_pivots:
+        bits, _ = O.allocate_bits_pivots(list(w.half_life[layer]), None, [4, 6, 8], w.avg_bits, w.n_pivots)
+        return np.asarray(bits, dtype=np.int32)
     bits, _ = O.allocate_bits_dp(list(w.half_life[layer]), None, [4, 6, 8], w.avg_bits)
     return np.asarray(bits, dtype=np.int32)
 
@@ -58,15 +63,32 @@ def ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ia - ib)
 
 
+def fp16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in binary16 ulps between two arrays of binary16 bit patterns (ordered
+    through zero: +0 and -0 coincide)."""
+    def key(h):
+        h = h.astype(np.int64)
+        return np.where(h & 0x8000, -(h & 0x7FFF), h)
+    return np.abs(key(a) - key(b))
+
+
 def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv=128) -> dict:
-    """Compare slot images [n, slot_stride] head by head."""
+    """Compare slot images [n, slot_stride] head by head (FP16 pivot heads by binary16 ulps)."""
     offs, stride = O.head_offsets(bits, dk, dv)
-    res = dict(max_code_diff=0, flips=0, elements=0, r_ulp=0, c_ulp=0, byte_equal=True)
+    res = dict(max_code_diff=0, flips=0, elements=0, r_ulp=0, c_ulp=0, byte_equal=True,
+               pivot_ulp=0, pivot_flips=0, pivot_elements=0)
     for s in range(gpu_bytes.shape[0]):
         for h, b in enumerate(bits):
             o = int(offs[h])
             n = O.block_bytes(int(b), dk, dv)
             g, r = gpu_bytes[s, o:o + n], ora_bytes[s, o:o + n]
+            if int(b) == 16:
+                d16 = fp16_ulp_diff(O.pivot_state(g, dk, dv), O.pivot_state(r, dk, dv))
+                res["pivot_ulp"] = max(res["pivot_ulp"], int(d16.max()))
+                res["pivot_flips"] += int((d16 > 0).sum())
+                res["pivot_elements"] += d16.size
+                res["byte_equal"] &= bool(np.array_equal(g, r))
+                continue
             if np.array_equal(g, r):
                 res["elements"] += dk * dv
                 continue
@@ -88,3 +110,11 @@ def y_max_rel(yg: np.ndarray, yo: np.ndarray) -> float:
     den = np.abs(yo).max(axis=-1)
     den = np.where(den > 0, den, 1.0)
     return float((num / den).max())
+
+
+def pivots_ok(res: dict) -> bool:
+    """The FP16 pivot bar: every binary16 value within PIVOT_ULP, off-by-one at a rate of at
+    most PIVOT_FLIP_RATE (fp32 kernel arithmetic against the fp64 oracle before rounding)."""
+    if res["pivot_elements"] == 0:
+        return True
+    return res["pivot_ulp"] <= PIVOT_ULP and res["pivot_flips"] <= max(1, PIVOT_FLIP_RATE * res["pivot_elements"])

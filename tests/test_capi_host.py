@@ -100,3 +100,20 @@ def test_allocator_candidate_order_and_errors(S):
         S.stepq_allocate_bits([1.0, -2.0], None, (4, 8), 6.0)  # negative half-life
     with pytest.raises(S.StepqError):
         S.stepq_allocate_bits([1.0], None, (4, 4), 6.0)        # duplicate candidate
+
+
+def test_pivot_allocator_equals_oracle(S):
+    """FP16 pivots: the C++ allocator picks the same pivot units and widths as the oracle's
+    ranking + exact DP, with and without a distortion table."""
+    rng = np.random.default_rng(60)
+    for trial in range(8):
+        N = [5, 8, 32, 32, 12, 3, 32, 7][trial]
+        npv = [1, 2, 1, 3, 0, 3, 2, 1][trial]
+        hl = np.exp(rng.uniform(0, math.log(4096), N))
+        dist = None if trial % 2 == 0 else rng.lognormal(0, 1, (N, 3)) * np.array([1, 0.1, 0.01])
+        ref, _ = O.allocate_bits_pivots(list(hl), dist, [4, 6, 8], 6.0, npv)
+        got = S.stepq_allocate_bits_pivots(hl, dist, (4, 6, 8), 6.0, npv)
+        assert list(got) == ref
+        assert int(np.sum(got == 16)) == npv
+    with pytest.raises(S.StepqError):
+        S.stepq_allocate_bits_pivots([1.0, 2.0], None, (4, 6, 8), 6.0, 3)    # more pivots than units

@@ -201,6 +201,45 @@ def test_decode_extreme_rows_vs_oracle(S):
     assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
 
 
+def test_pivot_heads_load_dump_and_step(S):
+    """FP16 pivot heads next to quantized heads: load = binary16 of the input (bit-exact),
+    dump exact, and one step (GDN fp32, KDA bf16) within the pivot bar and the usual bars."""
+    rng = np.random.default_rng(12)
+    bits = [16, 4, 16, 8]
+    n, H = 3, 4
+    st = random_states(rng, n, H)
+    ids = np.array([1, 4, 2], np.int32)
+    op = O.OraclePool(5, bits, H)
+    op.load_fp32(ids, st)
+    gp = S.Pool(5, bits, H, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    gp.load_fp32(slots_t(ids), dev(st))
+    gb, ob = dump_bytes(gp, ids), op.slot_bytes(ids)
+    off, _ = O.head_offsets(bits)
+    for s_ in range(n):
+        for h in (0, 2):
+            assert np.array_equal(O.pivot_state(gb[s_, off[h]:off[h] + 32768]),
+                                  st[s_, h].astype(np.float16).view(np.uint16))
+    out = torch.empty((n, H, 128, 128), dtype=torch.float32, device="cuda")
+    load_bytes(gp, ids, ob)
+    gp.dump_fp32(slots_t(ids), out)
+    assert np.array_equal(out.cpu().numpy(), op.dump_fp32(ids))
+    for gate, dtype, Hk in ((0, S.STEPQ_DTYPE_F32, H), (1, S.STEPQ_DTYPE_BF16, 2)):
+        op2 = O.OraclePool(5, bits, Hk, gate)
+        op2.load_fp32(ids, st)
+        x = dict(q=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)])),
+                 k=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)])),
+                 v=W.round_bf16(rng.standard_normal((n, H, 128)).astype(f32)),
+                 alpha=W.round_bf16(rng.uniform(0.6, 1, (n, H) if gate == 0 else (n, H, 128)).astype(f32)),
+                 beta=W.round_bf16(rng.uniform(0.1, 0.9, (n, H)).astype(f32)))
+        yg, sg, err = _run_gpu(S, bits, Hk, gate, dtype, x, op2.slot_bytes(ids), ids, 5)
+        yo = op2.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+        assert err == 0
+        res = PH.compare_slots(sg, op2.slot_bytes(ids), bits)
+        assert PH.pivots_ok(res), res
+        assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
+        assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
+
+
 def _run_gpu(S, bits, Hk, gate, dtype, x, init_bytes, ids, num_slots):
     gp = S.Pool(num_slots, bits, Hk, gate, dtype)
     load_bytes(gp, ids, init_bytes)
@@ -299,6 +338,9 @@ CASES = [
     (3, "mixed6", None, 0, 6, 64),
     (4, "mixed6", None, 0, 6, 64),
     (4, "uniform4", None, 0, 6, 32),
+    (4, "mixed6p", None, 0, 6, 32),
+    (3, "mixed6p", None, 0, 4, 32),
+    (2, "mixed6p", None, 0, 6, 32),
     (5, "mixed6", 64, 17, 3, 32),
     (5, "mixed6", 256, 17, 3, 32),
     (5, "mixed6", 1024, 0, 3, 32),
@@ -325,7 +367,8 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
     all_slots = slots_t(w.slot_ids)
     num = den = 0.0
     flips = elements = resyncs = 0
-    worst = dict(max_code_diff=0, r_ulp=0, c_ulp=0, y=0.0)
+    pflips = pelements = 0
+    worst = dict(max_code_diff=0, r_ulp=0, c_ulp=0, y=0.0, pivot_ulp=0)
     for t in range(steps):
         x = W.step_inputs(w, t, W.PHASE_RUN, layer)
         tx = PH.to_device(w, x, torch)
@@ -341,15 +384,19 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
         res = PH.compare_slots(gb, ob, bits)
         flips += res["flips"]
         elements += res["elements"]
-        for key in ("max_code_diff", "r_ulp", "c_ulp"):
+        pflips += res["pivot_flips"]
+        pelements += res["pivot_elements"]
+        for key in ("max_code_diff", "r_ulp", "c_ulp", "pivot_ulp"):
             worst[key] = max(worst[key], res[key])
         if not res["byte_equal"]:
             load_bytes(gp, sub_slots, ob)
             resyncs += 1
     assert gp.get_error() == 0
     rel = np.sqrt(num / den)
-    print("\n%s: y rel L2 %.3e, worst %s, flips %d / %d (%.2e), resyncs %d" %
-          (w.name, rel, worst, flips, elements, flips / elements, resyncs))
+    print("\n%s: y rel L2 %.3e, worst %s, flips %d / %d (%.2e), pivot flips %d / %d, resyncs %d" %
+          (w.name, rel, worst, flips, elements, flips / elements, pflips, pelements, resyncs))
+    assert worst["pivot_ulp"] <= PH.PIVOT_ULP
+    assert pflips <= max(1, PH.PIVOT_FLIP_RATE * pelements)
     assert worst["max_code_diff"] <= 1
     assert flips <= PH.CODE_FLIP_RATE * elements
     assert worst["r_ulp"] <= PH.R_ULP and worst["c_ulp"] <= PH.C_ULP
