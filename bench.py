@@ -47,6 +47,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--input-sets", type=int, default=N_INPUT_SETS,
                     help="distinct per-step input batches kept on the device and cycled")
+    ap.add_argument("--workload", default="pool", choices=["pool", "stack"],
+                    help="pool: the high-concurrency pool (the headline); stack: the 36-layer stack sweep")
+    ap.add_argument("--batch", type=int, default=1024, choices=[64, 256, 1024],
+                    help="requests of the stack sweep")
     return ap.parse_args()
 
 
@@ -222,10 +226,103 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def run_stack(args):
+    """36-layer stack sweep: a step runs layers 0..35 in order, each a decode step of its own
+    pool (per-layer allocation).  Timed twice on the device: 36 plain launches per step, and
+    the step captured once as a CUDA graph and replayed."""
+    import torch
+
+    from quantized_gated_delta_b200 import stepq
+    from quantized_gated_delta_b200 import workloads as W
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    w = W.make_workload(5, batch=args.batch)
+    L = w.layers
+    pools, bits_all = [], []
+    for layer in range(L):
+        bits = np.asarray(stepq.stepq_allocate_bits(w.half_life[layer], None, (4, 6, 8), w.avg_bits), np.uint8)
+        bits_all.append(bits)
+        pools.append(stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype))
+    slots = torch.from_numpy(w.slot_ids).cuda()
+
+    def dev_inputs(x):
+        return {k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).cuda() for k, v in x.items()}
+    nsets = 2
+    sets = [[dev_inputs(W.step_inputs(w, t, W.PHASE_RUN, layer)) for layer in range(L)] for t in range(nsets)]
+    y = torch.empty((w.B, w.H, w.dv), device="cuda")
+
+    def step(i):
+        xs = sets[i % nsets]
+        for layer in range(L):
+            x = xs[layer]
+            pools[layer].decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(0)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_plain = e0.elapsed_time(e1)
+    # the same step as one CUDA graph (inputs of set 0), replayed
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            step(0)
+    stream.wait_stream(side)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_graph = e0.elapsed_time(e1)
+    clocks = sampler.stop()
+    for p_ in pools:
+        if p_.get_error() != 0:
+            raise RuntimeError("device flag set in the stack sweep")
+    units = w.B * w.H * L * args.steps
+    value = units / (ms_graph / 1e3)
+    alg = sum(algorithmic_bytes_per_step(w, b) for b in bits_all)          # one step, all layers
+    peak, peak_kind = peaks()
+    achieved = alg * args.steps / (ms_graph / 1e3) / 1e9
+    line = {"metric": "quantized-state updates/s (req·head·layer-step), 36-layer stack", "value": value,
+            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_graph / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "%s: %d layers x H=%d, Hk=%d, B=%d, per-layer allocation (6.0 avg), bf16 inputs"
+                                   % (w.name, L, w.H, w.Hk, w.B),
+                       "pool_bytes": int(sum(p_.total_bytes for p_ in pools)),
+                       "l2": "no flush: each layer's pool is re-read after the other 35 (stack > 126 MB L2)"},
+            "us_per_layer_step_graph": ms_graph * 1e3 / (args.steps * L),
+            "us_per_layer_step_plain": ms_plain * 1e3 / (args.steps * L),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_kind, "traffic": None,
+                         "algorithmic_bytes_per_step": alg, "kernel": "decode_kernel (36 launches per step)"},
+            "gpu_launches": args.steps * L, "clocks": clocks}
+    print(json.dumps(line))
+    del g
+    for p_ in pools:
+        p_.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.workload == "stack":
+        run_stack(args)
         return
     import torch
 
