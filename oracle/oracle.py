@@ -61,8 +61,10 @@ def _load():
         "oracle_delta_step": (None, [I, I, P, P, P, P, P, F, P]),
         "oracle_step_state": (I, [I, I, I, P, P, P, P, P, P, P, F, P, P, P, P, P]),
         "oracle_head_offsets": (L, [I, P, I, I, P]),
-        "oracle_decode_step": (L, [I, I, I, I, I, P, I, P, P, I, P, P, P, P, P, P, I]),
-        "oracle_pool_load": (L, [I, I, I, P, I, P, P, I, P, I]),
+        "oracle_decode_step": (L, [I, I, I, I, I, P, I, P, P, I, P, P, P, P, P, P, I, P]),
+        "oracle_pool_load": (L, [I, I, I, P, I, P, P, I, P, I, P]),
+        "oracle_impact_normalize": (None, [I, P, P]),
+        "oracle_quantize_impact": (I, [I, I, I, P, P, P, P, P]),
         "oracle_pool_dump": (I, [I, I, I, P, I, P, P, I, P, I]),
         "oracle_fp_decode_step": (None, [I, I, I, I, I, I, P, P, P, P, P, P, P, I, I]),
         "oracle_fp16_encode": (None, [L, P, P]),
@@ -155,6 +157,25 @@ def pivot_state(blk: np.ndarray, dk: int = 128, dv: int = 128) -> np.ndarray:
     return _c(blk, np.uint8)[:2 * dk * dv].view(np.uint16).reshape(dk, dv).copy()
 
 
+def impact_normalize(omega) -> np.ndarray:
+    """Row-impact scores normalized to mean 1 (fp32 of the double quotient)."""
+    omega = _c(omega, np.float32)
+    w = np.zeros(omega.shape, dtype=np.float32)
+    _load().oracle_impact_normalize(len(omega), _p(omega), _p(w))
+    return w
+
+
+def quantize_impact(S32: np.ndarray, bits: int, w):
+    """Impact-weighted fit of an fp32 state with normalized weights w -> (Q, r, c, clipped)."""
+    S32 = _c(S32, np.float32)
+    dk, dv = S32.shape
+    Q = np.zeros((dk, dv), dtype=np.int32)
+    r = np.zeros(dk, dtype=np.float32)
+    c = np.zeros(dv, dtype=np.float32)
+    n = _load().oracle_quantize_impact(bits, dk, dv, _p(S32), _p(_c(w, np.float32)), _p(Q), _p(r), _p(c))
+    return Q, r, c, int(n)
+
+
 def make_block(Q, r, c, bits: int) -> np.ndarray:
     Q = _c(Q, np.int32)
     dk, dv = Q.shape
@@ -229,7 +250,7 @@ class OraclePool:
     binary16 values).  A zeroed pool is the zero state."""
 
     def __init__(self, num_slots: int, head_bits, num_key_heads: int, gate_mode: int = 0,
-                 dk: int = 128, dv: int = 128):
+                 dk: int = 128, dv: int = 128, impact=None):
         self.head_bits = _c(head_bits, np.int32)
         self.H = len(self.head_bits)
         self.Hk = int(num_key_heads)
@@ -240,6 +261,12 @@ class OraclePool:
         self.num_slots = int(num_slots)
         self.offsets, self.slot_stride = head_offsets(self.head_bits, dk, dv)
         self.data = np.zeros(self.num_slots * self.slot_stride, dtype=np.uint8)
+        # row-impact scores [H, dk] -> the impact-weighted fit for every quantized head
+        self.impact_w = None
+        if impact is not None:
+            impact = _c(impact, np.float32)
+            assert impact.shape == (self.H, dk) and (impact > 0).all()
+            self.impact_w = np.stack([impact_normalize(row) for row in impact])
 
     def block(self, slot: int, h: int) -> np.ndarray:
         o = slot * self.slot_stride + int(self.offsets[h])
@@ -264,7 +291,8 @@ class OraclePool:
         S = _c(S, np.float32)
         assert S.shape == (len(sl), self.H, self.dk, self.dv)
         rc = _load().oracle_pool_load(self.H, self.dk, self.dv, _p(self.head_bits), self.num_slots,
-                                      _p(self.data), _p(sl), len(sl), _p(S), nthreads or default_threads())
+                                      _p(self.data), _p(sl), len(sl), _p(S), nthreads or default_threads(),
+                                      None if self.impact_w is None else _p(self.impact_w))
         if rc < 0:
             raise IndexError("slot id out of range")
         return int(rc)
@@ -294,7 +322,8 @@ class OraclePool:
         rc = _load().oracle_decode_step(self.H, self.Hk, self.dk, self.dv, self.gate_mode,
                                         _p(self.head_bits), self.num_slots, _p(self.data), _p(sl), n,
                                         _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(y),
-                                        nthreads or default_threads())
+                                        nthreads or default_threads(),
+                                        None if self.impact_w is None else _p(self.impact_w))
         if rc < 0:
             raise IndexError("slot id out of range")
         if rc > 0:

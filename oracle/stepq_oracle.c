@@ -210,6 +210,75 @@ void oracle_dequantize(int dk, int dv, const int32_t *Q, const float *r, const f
 }
 
 /* ------------------------------------------------------------------------- */
+/* Key-row-aware dual-axis fit with row-impact scores ([SUM] Method para 4;    */
+/* [BLOG] offline vs per-step work)                                           */
+/* ------------------------------------------------------------------------- */
+/* Readings (the formulas did not survive): the row factor weighs the row's current
+ * magnitude against its impact with square-root scaling (a wider range for larger rows,
+ * finer resolution for higher-impact rows); the column scales are then fitted by the
+ * impact-weighted least-squares error, starting from the clip-free column scales of
+ * those rows; every entry goes to the nearest level.  One refit: from (c0, Q0) to
+ * c1 = the weighted least-squares scale of the codes Q0, then Q = the nearest levels
+ * under c1 (clipped to +-qmax).  Each half step can only lower the weighted error. */
+
+/* Row-impact weights normalized to mean 1: w_i = fp32(omega_i / mean(omega)), in double. */
+void oracle_impact_normalize(int dk, const float *omega, float *w)
+{
+    double sum = 0.0;
+    for (int i = 0; i < dk; i++) sum += (double)omega[i];
+    for (int i = 0; i < dk; i++) w[i] = (float)((double)omega[i] / (sum / dk));
+}
+
+/* Fit and quantize an fp32 state with normalized row-impact weights w (all > 0):
+ *   m_i  = max_j |S_ij|;   r_i = fp32(sqrt(m_i / w_i))
+ *   c0_j = fp32(max_{i: r_i > 0} (|S_ij| / r_i) / qmax)
+ *   Q0   = nearest level of S / (r c0)
+ *   c1_j = fp32(sum_i w_i r_i Q0_ij S_ij / sum_i w_i r_i^2 Q0_ij^2), or c0_j when either
+ *          sum is not positive
+ *   Q    = nearest level of S / (r c1), clipped to [-qmax, qmax]
+ * Returns the number of codes the final clip moved. */
+int oracle_quantize_impact(int bits, int dk, int dv, const float *S32, const float *w, int32_t *Q, float *r, float *c)
+{
+    const int qmax = oracle_qmax(bits);
+    int clipped = 0;
+    for (int i = 0; i < dk; i++) {
+        double m = 0.0;
+        for (int j = 0; j < dv; j++) {
+            double a = fabs((double)S32[(long)i * dv + j]);
+            if (a > m) m = a;
+        }
+        r[i] = (float)sqrt(m / (double)w[i]);
+    }
+    for (int j = 0; j < dv; j++) {
+        double mx = 0.0;
+        for (int i = 0; i < dk; i++)
+            if (r[i] > 0.0f) {
+                double t = fabs((double)S32[(long)i * dv + j]) / (double)r[i];
+                if (t > mx) mx = t;
+            }
+        const float c0 = (float)(mx / (double)qmax);
+        double num = 0.0, den = 0.0;
+        for (int i = 0; i < dk; i++) {
+            double scale = (double)r[i] * (double)c0;
+            double q0 = scale > 0.0 ? nearbyint((double)S32[(long)i * dv + j] / scale) : 0.0;
+            if (q0 > qmax) q0 = qmax;
+            if (q0 < -qmax) q0 = -qmax;
+            num += (double)w[i] * (double)r[i] * q0 * (double)S32[(long)i * dv + j];
+            den += (double)w[i] * (double)r[i] * (double)r[i] * q0 * q0;
+        }
+        c[j] = (num > 0.0 && den > 0.0) ? (float)(num / den) : c0;
+        for (int i = 0; i < dk; i++) {
+            double scale = (double)r[i] * (double)c[j];
+            double qv = scale > 0.0 ? nearbyint((double)S32[(long)i * dv + j] / scale) : 0.0;
+            if (qv > qmax) { qv = qmax; clipped++; }
+            if (qv < -qmax) { qv = -qmax; clipped++; }
+            Q[(long)i * dv + j] = (int32_t)qv;
+        }
+    }
+    return clipped;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Gated Delta-rule step ([EXP] mechanism)                                    */
 /* ------------------------------------------------------------------------- */
 
@@ -251,9 +320,33 @@ void oracle_delta_step(int dk, int dv, double *S, const float *q, const float *k
  * dequantize -> delta step -> readout -> round the state to fp32 -> fit -> quantize.
  * S_pre (optional, [dk*dv]) receives the updated state before quantization (double).
  * Returns the clip count of the fit (0 expected). */
+static int step_state_fit(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
+                          const float *q, const float *k, const float *v, const float *alpha, float beta,
+                          int32_t *Q_out, float *r_out, float *c_out, float *y_out, double *S_pre,
+                          const float *impact);
+
 int oracle_step_state(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
                       const float *q, const float *k, const float *v, const float *alpha, float beta,
                       int32_t *Q_out, float *r_out, float *c_out, float *y_out, double *S_pre)
+{
+    return step_state_fit(dk, dv, bits, Q_in, r_in, c_in, q, k, v, alpha, beta, Q_out, r_out, c_out, y_out,
+                          S_pre, NULL);
+}
+
+/* The same step with the impact-weighted fit (normalized weights w[dk]); returns the number
+ * of codes its final clip moved (legitimate for this fit). */
+int oracle_step_state_impact(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
+                             const float *q, const float *k, const float *v, const float *alpha, float beta,
+                             const float *w, int32_t *Q_out, float *r_out, float *c_out, float *y_out)
+{
+    return step_state_fit(dk, dv, bits, Q_in, r_in, c_in, q, k, v, alpha, beta, Q_out, r_out, c_out, y_out,
+                          NULL, w);
+}
+
+static int step_state_fit(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
+                          const float *q, const float *k, const float *v, const float *alpha, float beta,
+                          int32_t *Q_out, float *r_out, float *c_out, float *y_out, double *S_pre,
+                          const float *impact)
 {
     long ne = (long)dk * dv;
     double *S = (double *)malloc((size_t)ne * sizeof(double));
@@ -264,7 +357,8 @@ int oracle_step_state(int dk, int dv, int bits, const int32_t *Q_in, const float
     for (int j = 0; j < dv; j++) y_out[j] = (float)y[j];
     if (S_pre) memcpy(S_pre, S, (size_t)ne * sizeof(double));
     for (long e = 0; e < ne; e++) S32[e] = (float)S[e];
-    int clipped = oracle_quantize(bits, dk, dv, S32, Q_out, r_out, c_out);
+    int clipped = impact ? oracle_quantize_impact(bits, dk, dv, S32, impact, Q_out, r_out, c_out)
+                         : oracle_quantize(bits, dk, dv, S32, Q_out, r_out, c_out);
     free(S); free(y); free(S32);
     return clipped;
 }
@@ -307,12 +401,13 @@ static void write_block(uint8_t *blk, int bits, int dk, int dv, const int32_t *Q
  *   q, k      [n, Hk, dk]; v [n, H, dv]; beta [n, H]
  *   alpha     gate_mode 0 (GDN): [n, H];  gate_mode 1 (KDA): [n, H, dk]
  *   y         [n, H, dv] (fp32 out)
- * Value head h reads key head h / (H / Hk).  Returns the total clip count, or -1
- * for an out-of-range slot id (that request is skipped). */
+ *   impact    NULL (clip-free fit) or [H, dk] normalized row-impact weights (impact fit)
+ * Value head h reads key head h / (H / Hk).  Returns the clip count of the clip-free fit
+ * (0 when it holds), or -1 for an out-of-range slot id (that request is skipped). */
 long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int32_t *head_bits,
                         int num_slots, uint8_t *pool, const int32_t *slot_ids, int n,
                         const float *q, const float *k, const float *v, const float *alpha,
-                        const float *beta, float *y, int nthreads)
+                        const float *beta, float *y, int nthreads, const float *impact)
 {
     long *offsets = (long *)malloc((size_t)H * sizeof(long));
     long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
@@ -352,10 +447,16 @@ long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int3
         read_block(blk, bits, dk, dv, Q, r, c);
         for (int i = 0; i < dk; i++)
             al[i] = gate_mode == 0 ? alpha[(long)b * H + h] : alpha[((long)b * H + h) * dk + i];
-        clipped += oracle_step_state(dk, dv, bits, Q, r, c,
-                                     q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
-                                     v + ((long)b * H + h) * dv, al, beta[(long)b * H + h],
-                                     Q2, r2, c2, y + ((long)b * H + h) * dv, NULL);
+        if (impact)
+            (void)oracle_step_state_impact(dk, dv, bits, Q, r, c, q + ((long)b * Hk + g) * dk,
+                                           k + ((long)b * Hk + g) * dk, v + ((long)b * H + h) * dv, al,
+                                           beta[(long)b * H + h], impact + (long)h * dk, Q2, r2, c2,
+                                           y + ((long)b * H + h) * dv);
+        else
+            clipped += oracle_step_state(dk, dv, bits, Q, r, c,
+                                         q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
+                                         v + ((long)b * H + h) * dv, al, beta[(long)b * H + h],
+                                         Q2, r2, c2, y + ((long)b * H + h) * dv, NULL);
         write_block(blk, bits, dk, dv, Q2, r2, c2);
         free(Q); free(Q2); free(r); free(c); free(r2); free(c2); free(al);
     }
@@ -363,9 +464,10 @@ long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int3
     return bad ? -1 : clipped;
 }
 
-/* Quantize fp32 states S [n, H, dk, dv] into the slots slot_ids[n] of a pool. */
+/* Quantize fp32 states S [n, H, dk, dv] into the slots slot_ids[n] of a pool (impact: as for
+ * oracle_decode_step). */
 long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_slots, uint8_t *pool,
-                      const int32_t *slot_ids, int n, const float *S, int nthreads)
+                      const int32_t *slot_ids, int n, const float *S, int nthreads, const float *impact)
 {
     long *offsets = (long *)malloc((size_t)H * sizeof(long));
     long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
@@ -387,7 +489,10 @@ long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_s
         }
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
-        clipped += oracle_quantize(head_bits[h], dk, dv, S + it * ne, Q, r, c);
+        if (impact)
+            (void)oracle_quantize_impact(head_bits[h], dk, dv, S + it * ne, impact + (long)h * dk, Q, r, c);
+        else
+            clipped += oracle_quantize(head_bits[h], dk, dv, S + it * ne, Q, r, c);
         write_block(pool + (long)slot * stride + offsets[h], head_bits[h], dk, dv, Q, r, c);
         free(Q); free(r); free(c);
     }
