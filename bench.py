@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--input-sets", type=int, default=N_INPUT_SETS,
                     help="distinct per-step input batches kept on the device and cycled")
+    ap.add_argument("--fit", default="clipfree", choices=["clipfree", "impact"],
+                    help="dual-axis fit: clip-free (the headline) or impact-weighted with synthetic row-impact scores")
     ap.add_argument("--workload", default="pool", choices=["pool", "stack"],
                     help="pool: the high-concurrency pool (the headline); stack: the 36-layer stack sweep")
     ap.add_argument("--batch", type=int, default=1024, choices=[64, 256, 1024],
@@ -344,6 +346,8 @@ def main():
         bits = stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
     bits = np.asarray(bits, dtype=np.uint8)
     pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    if args.fit == "impact":
+        pool.set_impact(W.impact_scores(w))
     slots = torch.from_numpy(w.slot_ids).cuda()
 
     # per-step inputs, resident in HBM (bf16 bit patterns)
@@ -435,9 +439,10 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s"
+            "config": {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s%s"
                        % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
-                          "".join(str(int(b)) for b in bits)),
+                          "".join(str(int(b)) for b in bits),
+                          ", impact-weighted fit" if args.fit == "impact" else ""),
                        "avg_bits": float(np.mean(bits)), "parallelism": "dp%d (independent pools)" % world,
                        "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
                              % (w.B * sum(block_bytes(int(b)) for b in bits) / 1e6),

@@ -167,6 +167,20 @@ STEPQ_API int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *st
                                         const void *alpha, const void *beta, float *y, int32_t *flag_out,
                                         stepq_stream stream);
 
+/* Key-row-aware dual-axis fitting with row-impact scores.          [SUM Method, paras 3-4; BLOG]
+ * impact: HOST [H, d_k] float32 row-impact scores (positive, finite; fixed offline, e.g. the
+ * expected squared readout weight of each key row over calibration tokens), or NULL to
+ * return to the clip-free fit.  Each head's scores are normalized to mean 1
+ * (w_i = float(omega_i / mean(omega)), in double).  While set, stepq_pool_load_fp32 and
+ * stepq_decode_step fit every quantized head of the pool as (S: the updated state in fp32):
+ *   r_i  = sqrt(max_j |S_ij| / w_i)                      row: magnitude against impact
+ *   c0_j = max_i (|S_ij| / r_i) / qmax,  Q0 = nearest levels of S / (r c0)
+ *   c_j  = sum_i w_i r_i Q0_ij S_ij / sum_i w_i r_i^2 Q0_ij^2   (c0_j if a sum is <= 0)
+ *   Q    = nearest levels of S / (r c), clipped to [-qmax, qmax]
+ * FP16 pivot heads are unaffected.  Synchronizes the device; STEPQ_INVALID_ARG for a
+ * non-positive or non-finite score. */
+STEPQ_API int stepq_pool_set_impact(stepq_pool *pool, const float *impact);
+
 /* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
  * Synchronizes the device. */
 STEPQ_API int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out);

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "stepq_internal.h"
 #include "stepq_tile.cuh"
@@ -47,6 +48,7 @@ void free_pool(stepq_pool *p)
     cudaFree(p->d_bits);
     cudaFree(p->d_order);
     cudaFree(p->d_flag);
+    cudaFree(p->d_impact);
     delete p;
 }
 
@@ -207,6 +209,38 @@ int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, cons
     if (pool->gate_mode == STEPQ_GATE_KDA ? !aligned16(alpha) : !aligned_to(alpha, esz)) return STEPQ_INVALID_ARG;
     if (!aligned_to(beta, esz)) return STEPQ_INVALID_ARG;
     return status_of(stepq::launch_decode(pool, slot_ids, n, q, k, v, alpha, beta, y, stream));
+}
+
+int stepq_pool_set_impact(stepq_pool *pool, const float *impact)
+{
+    if (!pool) return STEPQ_INVALID_ARG;
+    int st = check_device(pool);
+    if (st != STEPQ_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();           // no launch in flight reads the table
+    if (e != cudaSuccess) return status_of(e);
+    if (!impact) {
+        e = cudaFree(pool->d_impact);
+        pool->d_impact = nullptr;
+        return status_of(e);
+    }
+    const int n = pool->H * stepq::DK;
+    std::vector<float> w(size_t(n), 0.0f);
+    for (int h = 0; h < pool->H; ++h) {
+        double sum = 0.0;
+        for (int i = 0; i < stepq::DK; ++i) {
+            const float o = impact[h * stepq::DK + i];
+            if (!(o > 0.0f) || !(o < 3.0e38f)) return STEPQ_INVALID_ARG;     // positive and finite
+            sum += double(o);
+        }
+        for (int i = 0; i < stepq::DK; ++i)
+            w[size_t(h) * stepq::DK + i] = float(double(impact[h * stepq::DK + i]) / (sum / stepq::DK));
+    }
+    if (!pool->d_impact) {
+        e = cudaMalloc(&pool->d_impact, sizeof(float) * size_t(n));
+        if (e != cudaSuccess) return status_of(e);
+    }
+    e = cudaMemcpy(pool->d_impact, w.data(), sizeof(float) * size_t(n), cudaMemcpyHostToDevice);
+    return status_of(e);
 }
 
 int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out)

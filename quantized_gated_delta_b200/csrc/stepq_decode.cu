@@ -65,6 +65,7 @@ struct DecodeArgs {
     int num_slots, H, Hk, group;
     int nh4, nh6;                   // heads of width 4 and 6 (visited first, in that order)
     int Hq;                         // quantized heads: the first Hq entries of head_order
+    const float *impact;            // [H, d_k] normalized row-impact weights (impact fit), or null
     const int32_t *slot_ids;
     int n;
     int step_b, step_h;             // gridDim.x in head-major items = step_h * n + step_b
@@ -81,6 +82,7 @@ struct Scratch {
     float4 whi[DK];                 // per row {rho q, rho q, rho k, rho k}  (lanes 16..31)
     float4 wrk[DK];                 // per row {rho, rho, k, k}
     float2 ir[DK];                  // per row {1/r, 1/r}
+    float4 fit[DK];                 // impact fit, per row {1/r, 1/r, w r^2, w r^2}
     float xd[NPANEL * PANEL];       // d_j / c'_j per column
     float xg[NPANEL * PANEL];       // c'_j / c_new_j per column
     float kqw[4];                   // partial k.q of the next state (warps 4..7)
@@ -137,6 +139,12 @@ __device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs
 // next row table, then quantization, packing and the per-warp stores.  Returns false on
 // every thread when some thread saw a failed wait.
 template <int GATE, typename TIn, int BITS>
+__device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *stages, int i, bool has_next,
+                                             const DecodeArgs &a, Scratch &sc, const TileIdx<4> &ix, int tid, int h,
+                                             float cprime, TIn alpha_next_raw, bool ok, float *r_io, float *c_io,
+                                             uint8_t *codes);
+
+template <int GATE, typename TIn, int BITS, bool IMPACT>
 __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_next, const DecodeArgs &a, Scratch &sc,
                                             const TileIdx<4> &ix, int tid, long long bh, float beta, float kq,
                                             TIn alpha_next_raw, bool ok)
@@ -223,6 +231,9 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
             T[m][j + 1] = t.y;
         }
     }
+    if constexpr (IMPACT)
+        return refit_impact<GATE, TIn, BITS>(T, stages, i, has_next, a, sc, ix, tid, int(bh % a.H), cprime,
+                                             alpha_next_raw, ok, r_io, c_io, codes);
     // column maxima: over the thread's rows, then a warp-wide max per column; the 16
     // results go through shared memory (the d' buffer, already read) to the column lanes
 #pragma unroll
@@ -319,9 +330,153 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     return true;
 }
 
+// Key-row-aware dual-axis fit with row-impact weights (STEPQuant summary, "Method" para 4):
+// on entry T_ij = S_ij / c'_j.  r_i = sqrt(max_j |S_ij| / w_i); c0_j = max_i |S_ij / r_i| / qmax;
+// Q0 = nearest levels of S / (r c0); c_j = sum_i w_i r_i Q0_ij S_ij / sum_i w_i r_i^2 Q0_ij^2
+// (c0_j when a sum is not positive); codes = nearest levels of S / (r c), clipped.  With
+// P_ij = S_ij / r_i the sums are sum (w r^2) Q0 P and sum (w r^2) Q0^2, reduced over the warp
+// like the column dot products.
+template <int GATE, typename TIn, int BITS>
+__device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *stages, int i, bool has_next,
+                                             const DecodeArgs &a, Scratch &sc, const TileIdx<4> &ix, int tid, int h,
+                                             float cprime, TIn alpha_next_raw, bool ok, float *r_io, float *c_io,
+                                             uint8_t *codes)
+{
+    constexpr int QM = qmax_of(BITS);
+    constexpr float MAG = kTwo23 + float(1 << (BITS - 1));
+    const int lane = ix.lane;
+    const int panel = ix.panel;
+    const bool upper = (lane & 16) != 0;
+    const int col = lane & 15;
+    float *cbuf = sc.xg + panel * PANEL;            // one value per column of the panel
+
+    // S_ij = c'_j T_ij, and the thread's row maxima of |S| (panel partials)
+    st_shared_if(!upper, cbuf + col, cprime);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        const float4 cp = *reinterpret_cast<const float4 *>(cbuf + j);
+#pragma unroll
+        for (int m = 0; m < kRows; ++m) {
+            const float2 x = fmul2(make_float2(T[m][j], T[m][j + 1]), make_float2(cp.x, cp.y));
+            const float2 z = fmul2(make_float2(T[m][j + 2], T[m][j + 3]), make_float2(cp.z, cp.w));
+            T[m][j] = x.x; T[m][j + 1] = x.y; T[m][j + 2] = z.x; T[m][j + 3] = z.y;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+        float mx = absmax3(T[m][0], T[m][1], T[m][2]);
+#pragma unroll
+        for (int j = 3; j < PANEL - 1; j += 2) mx = absmax3(mx, T[m][j], T[m][j + 1]);
+        mx = fmaxf(mx, fabsf(T[m][PANEL - 1]));
+        sc.rp[ix.row(m) * kRpStride + panel] = mx;
+    }
+    if (__syncthreads_or(!ok)) return false;
+
+    // ---- threads 0..127: r, 1/r and w r^2 of row tid (IEEE sqrt and divide; r is normal);
+    //      threads 128..255: the next state's row weights
+    if (tid < DK) {
+        const float4 u = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride);
+        const float4 v = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride + 4);
+        const float mr = fmaxf(max3(u.x, u.y, u.z), max3(max3(u.w, v.x, v.y), v.z, v.w));
+        const float w = a.impact[h * DK + tid];
+        const float r = __fsqrt_rn(__fdiv_rn(mr, w));
+        r_io[tid] = r;
+        const float ir = r > 0.0f ? __frcp_rn(r) : 0.0f;
+        const float wr2 = w * r * r;
+        sc.fit[tid] = make_float4(ir, ir, wr2, wr2);
+        fence_proxy_async_smem();                  // r is bulk-stored from the stage by warp 0
+    } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
+        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
+                             to_f32(alpha_next_raw), sc, tid);
+    }
+    __syncthreads();
+
+    // ---- P_ij = S_ij / r_i; column maxima of |P| give c0 = max / qmax
+    float2 wr[kRows];
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+        const float4 f = sc.fit[ix.row(m)];
+        wr[m] = make_float2(f.z, f.w);
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            const float2 p = fmul2(make_float2(T[m][j], T[m][j + 1]), make_float2(f.x, f.y));
+            T[m][j] = p.x;
+            T[m][j + 1] = p.y;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        float cm[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            cm[e] = warp_absmax(fmaxf(absmax3(T[0][j + e], T[1][j + e], T[2][j + e]), fabsf(T[3][j + e])));
+        st_shared_v4_if(lane == 0, sc.xd + panel * PANEL + j, make_float4(cm[0], cm[1], cm[2], cm[3]));
+    }
+    __syncwarp();
+    const float c0 = div_const<QM>(sc.xd[panel * PANEL + col]);
+    st_shared_if(!upper, cbuf + col, c0 > 0.0f ? rcp_refined(c0) : 0.0f);
+    __syncwarp();
+
+    // ---- codes Q0 under c0 and the weighted least-squares sums of each column: lanes 0..15
+    // keep the numerators after the first reduce step, lanes 16..31 the denominators
+    float A[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 2) {
+        const float2 ic = *reinterpret_cast<const float2 *>(cbuf + j);
+        float2 sn = make_float2(0.0f, 0.0f), sd = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int m = 0; m < kRows; ++m) {
+            const float2 p = make_float2(T[m][j], T[m][j + 1]);
+            const float2 q0 = fadd2(ffma2(p, ic, make_float2(MAG, MAG)), make_float2(-MAG, -MAG));
+            const float2 z = fmul2(q0, wr[m]);
+            sn = ffma2(z, p, sn);
+            sd = ffma2(z, q0, sd);
+        }
+        A[j] = (upper ? sd.x : sn.x) + __shfl_xor_sync(kFull, upper ? sn.x : sd.x, 16);
+        A[j + 1] = (upper ? sd.y : sn.y) + __shfl_xor_sync(kFull, upper ? sn.y : sd.y, 16);
+    }
+    reduce_scatter<PANEL, 4, 8, false>(A, lane);
+    const float other = __shfl_xor_sync(kFull, A[0], 16);
+    const float num = upper ? other : A[0], den = upper ? A[0] : other;
+    const float c1 = (num > 0.0f && den > 0.0f) ? div_refined(num, den) : c0;
+    st_shared_if(!upper, c_io + panel * PANEL + col, c1);
+    st_shared_if(!upper, cbuf + col, c1 > 0.0f ? rcp_refined(c1) : 0.0f);
+    __syncwarp();
+    float icl[PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; j += 4) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(cbuf + j);
+        icl[j] = t4.x; icl[j + 1] = t4.y; icl[j + 2] = t4.z; icl[j + 3] = t4.w;
+    }
+
+    // ---- codes = nearest levels of P / c, clipped to [-qmax, qmax]
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+        uint32_t u[PANEL];
+#pragma unroll
+        for (int j = 0; j < PANEL; j += 2) {
+            const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(icl[j], icl[j + 1]),
+                                   make_float2(MAG, MAG));
+            u[j] = __float_as_uint(fminf(fmaxf(f.x, MAG - float(QM)), MAG + float(QM)));
+            u[j + 1] = __float_as_uint(fminf(fmaxf(f.y, MAG - float(QM)), MAG + float(QM)));
+        }
+        pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + ix.row(m) * seg_bytes(BITS));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        uint8_t *dst = a.pool + sc.meta[i % kStages].dst;
+        bulk_s2g(dst + panel * panel_bytes(BITS), codes + panel * panel_bytes(BITS), panel_bytes(BITS));
+        bulk_s2g(dst + codes_bytes(BITS) + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
+        if (panel == 0) bulk_s2g(dst + codes_bytes(BITS), r_io, 4 * DK);
+    }
+    return true;
+}
+
 // Per-CTA state of the item loop.  The loop runs in three pieces, one per bit width
 // (the heads are visited grouped by width), so each piece is compiled for one width.
-template <int GATE, typename TIn>
+template <int GATE, typename TIn, bool IMPACT>
 struct ItemLoop {
     const DecodeArgs &a;
     Scratch &sc;
@@ -420,7 +575,7 @@ struct ItemLoop {
                     __syncthreads();
                 }
             } else {
-                alive = decode_item<GATE, TIn, BITS>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
+                alive = decode_item<GATE, TIn, BITS, IMPACT>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
                                                      alpha_raw, ok);
             }
             if (!alive) return false;
@@ -433,7 +588,7 @@ struct ItemLoop {
     }
 };
 
-template <int GATE, typename TIn>
+template <int GATE, typename TIn, bool IMPACT>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -468,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     }
     __syncthreads();
 
-    ItemLoop<GATE, TIn> L(a, sc, stages, tid, count);
+    ItemLoop<GATE, TIn, IMPACT> L(a, sc, stages, tid, count);
     L.cur = {int(first % a.n), int(first / a.n)};
     if (tid == 0) {
         sc.prod_b = L.cur.b;
@@ -633,14 +788,19 @@ size_t decode_smem_max()
 template <int GATE, typename TIn>
 cudaError_t configure_one(stepq_pool *p)
 {
-    auto kern = decode_kernel<GATE, TIn>;
+    auto kern = decode_kernel<GATE, TIn, false>;
+    auto kern_impact = decode_kernel<GATE, TIn, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern_impact, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
+    int per_sm = 0, per_sm_impact = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, p->decode_smem);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_impact, kern_impact, kThreads, p->decode_smem);
     if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    p->decode_grid = per_sm * p->num_sms;
+    if (per_sm < 1 || per_sm_impact < 1) return cudaErrorInvalidConfiguration;
+    p->decode_grid = (per_sm < per_sm_impact ? per_sm : per_sm_impact) * p->num_sms;
     return cudaSuccess;
 }
 
@@ -701,6 +861,7 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.blk_cap = p->blk_cap;
     a.stage_bytes = p->stage_bytes;
     a.Hq = p->H - p->npiv;
+    a.impact = p->d_impact;
     // items are dealt round-robin in head-major order, so the CTAs resident at any moment
     // work on one or two heads (one bit width: one code path in the instruction caches)
     const long long total = (long long)n * a.Hq;
@@ -708,16 +869,29 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
         const int grid = int(total < p->decode_grid ? total : p->decode_grid);
         a.step_b = grid % n;
         a.step_h = grid / n;
-        if (p->gate_mode == STEPQ_GATE_GDN) {
+        const size_t sm = p->decode_smem;
+        if (a.impact) {
+            if (p->gate_mode == STEPQ_GATE_GDN) {
+                if (p->in_dtype == STEPQ_DTYPE_BF16)
+                    decode_kernel<STEPQ_GATE_GDN, uint16_t, true><<<grid, kThreads, sm, stream>>>(a);
+                else
+                    decode_kernel<STEPQ_GATE_GDN, float, true><<<grid, kThreads, sm, stream>>>(a);
+            } else {
+                if (p->in_dtype == STEPQ_DTYPE_BF16)
+                    decode_kernel<STEPQ_GATE_KDA, uint16_t, true><<<grid, kThreads, sm, stream>>>(a);
+                else
+                    decode_kernel<STEPQ_GATE_KDA, float, true><<<grid, kThreads, sm, stream>>>(a);
+            }
+        } else if (p->gate_mode == STEPQ_GATE_GDN) {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                decode_kernel<STEPQ_GATE_GDN, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+                decode_kernel<STEPQ_GATE_GDN, uint16_t, false><<<grid, kThreads, sm, stream>>>(a);
             else
-                decode_kernel<STEPQ_GATE_GDN, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+                decode_kernel<STEPQ_GATE_GDN, float, false><<<grid, kThreads, sm, stream>>>(a);
         } else {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                decode_kernel<STEPQ_GATE_KDA, uint16_t><<<grid, kThreads, p->decode_smem, stream>>>(a);
+                decode_kernel<STEPQ_GATE_KDA, uint16_t, false><<<grid, kThreads, sm, stream>>>(a);
             else
-                decode_kernel<STEPQ_GATE_KDA, float><<<grid, kThreads, p->decode_smem, stream>>>(a);
+                decode_kernel<STEPQ_GATE_KDA, float, false><<<grid, kThreads, sm, stream>>>(a);
         }
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -787,13 +961,13 @@ cudaError_t noalloc_setup(int dev, NoallocDevice **out)
         e = upload_tables();
         if (e != cudaSuccess) return e;
         const int smem = int(decode_smem_max());
-        e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, uint16_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, uint16_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         d.scratch = static_cast<uint8_t *>(ptr);
         d.ready = true;
@@ -807,7 +981,7 @@ cudaError_t noalloc_launch(const DecodeArgs &a0, int num_sms, size_t smem, cudaS
 {
     DecodeArgs a = a0;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<GATE, TIn>, kThreads, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<GATE, TIn, false>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long total = (long long)a.n * a.H;
@@ -815,7 +989,7 @@ cudaError_t noalloc_launch(const DecodeArgs &a0, int num_sms, size_t smem, cudaS
     const int grid = int(total < cap ? total : cap);
     a.step_b = grid % a.n;
     a.step_h = grid / a.n;
-    decode_kernel<GATE, TIn><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<GATE, TIn, false><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -884,6 +1058,7 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     a.Hk = desc->num_key_heads;
     a.group = H / desc->num_key_heads;
     a.Hq = H;
+    a.impact = nullptr;
     count_widths(bits, H, a);
     a.slot_ids = slot_ids;
     a.n = n;

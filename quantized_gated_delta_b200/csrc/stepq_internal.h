@@ -22,6 +22,7 @@ struct stepq_pool {
     uint8_t *d_bits = nullptr;          // [H]
     int32_t *d_order = nullptr;         // [H] head processing order (widths 4, 6, 8, then pivots)
     int *d_flag = nullptr;              // sticky device flag (STEPQ_FLAG_* bits)
+    float *d_impact = nullptr;          // [H, d_k] normalized row-impact weights (impact fit), or null
     int decode_grid = 0;                // persistent CTAs for the decode kernel
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel
     int stage_bytes = 0;

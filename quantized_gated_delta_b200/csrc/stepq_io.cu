@@ -113,6 +113,73 @@ __device__ __forceinline__ bool fit_quantize_pack(float (&S)[ROWS][PANEL], const
 }
 
 // ------------------------------------------------------------------------------------------
+// The impact-weighted fit (STEPQuant summary, "Method" para 4) of a register tile, in the
+// order of its definition and with IEEE division and square root (w: the head's normalized
+// row-impact weights):  r_i = sqrt(max_j |S_ij| / w_i);  c0_j = max_i |S_ij / r_i| / qmax;
+// Q0 = nearest levels of S / (r c0);  c_j = sum_i w_i r_i Q0_ij S_ij / sum_i w_i r_i^2 Q0_ij^2
+// (c0_j when a sum is not positive);  codes = nearest levels of S / (r c), clipped.
+// ------------------------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ void fit_quantize_pack_impact(float (&S)[4][PANEL], const TileIdx<4> &ix, float *rp,
+                                                         const float *w, uint8_t *codes_out, float *r_out,
+                                                         float *c_out)
+{
+    constexpr int QM = qmax_of(BITS);
+    // row maxima of |S| over the panels
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        float a = absmax3(S[m][0], S[m][1], S[m][2]);
+#pragma unroll
+        for (int j = 3; j < PANEL; j += 2)
+            a = (j + 1 < PANEL) ? absmax3(a, S[m][j], S[m][j + 1]) : fmaxf(a, fabsf(S[m][j]));
+        rp[ix.row(m) * kIoRpStride + ix.panel] = a;
+    }
+    __syncthreads();
+    float r[4], P[4][PANEL];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int row = ix.row(m);
+        const float4 a = *reinterpret_cast<const float4 *>(rp + row * kIoRpStride);
+        const float4 b = *reinterpret_cast<const float4 *>(rp + row * kIoRpStride + 4);
+        const float mr = max3(max3(a.x, a.y, a.z), max3(a.w, b.x, b.y), fmaxf(b.z, b.w));
+        r[m] = sqrtf(mr / w[row]);
+        if (ix.panel == 0) r_out[row] = r[m];
+#pragma unroll
+        for (int j = 0; j < PANEL; ++j) P[m][j] = r[m] > 0.0f ? S[m][j] / r[m] : 0.0f;
+    }
+    // per column (the warp holds all 128 rows of its panel): c0, the sums, c
+    uint32_t u[4][PANEL];
+#pragma unroll
+    for (int j = 0; j < PANEL; ++j) {
+        const float mx = warp_absmax(fmaxf(absmax3(P[0][j], P[1][j], P[2][j]), fabsf(P[3][j])));
+        const float c0 = mx / float(QM);
+        float num = 0.0f, den = 0.0f;
+        float q0[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            q0[m] = c0 > 0.0f ? fminf(fmaxf(rintf(P[m][j] / c0), -float(QM)), float(QM)) : 0.0f;
+            const float wr = w[ix.row(m)] * r[m];
+            num = fmaf(wr * q0[m], S[m][j], num);
+            den = fmaf(wr * r[m] * q0[m], q0[m], den);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            num += __shfl_xor_sync(0xffffffffu, num, o);
+            den += __shfl_xor_sync(0xffffffffu, den, o);
+        }
+        const float c = (num > 0.0f && den > 0.0f) ? num / den : c0;
+        if (ix.lane == 0) c_out[ix.panel * PANEL + j] = c;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float q = c > 0.0f ? fminf(fmaxf(rintf(P[m][j] / c), -float(QM)), float(QM)) : 0.0f;
+            u[m][j] = __float_as_uint(q + (kTwo23 + float(1 << (BITS - 1))));
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) pack_seg<BITS>(u[m], codes_out + ix.panel * panel_bytes(BITS) + ix.row(m) * seg_bytes(BITS));
+}
+
+// ------------------------------------------------------------------------------------------
 // Pool I/O kernels: one CTA (256 threads, 4 x 16 tiles) per (request, head) state.
 // ------------------------------------------------------------------------------------------
 struct IoArgs {
@@ -123,11 +190,12 @@ struct IoArgs {
     int num_slots, H;
     const int32_t *slot_ids;
     int *flag;
+    const float *impact;            // [H, d_k] normalized row-impact weights, or null (clip-free fit)
 };
 
 template <int BITS>
 __device__ __forceinline__ void load_fp32_item(const IoArgs &a, uint8_t *blk, const float *S,
-                                               const TileIdx<4> &ix, float *rp, float *xc)
+                                               const TileIdx<4> &ix, float *rp, float *xc, int h)
 {
     float T[4][PANEL];
 #pragma unroll
@@ -138,7 +206,10 @@ __device__ __forceinline__ void load_fp32_item(const IoArgs &a, uint8_t *blk, co
             T[m][j] = t.x; T[m][j + 1] = t.y; T[m][j + 2] = t.z; T[m][j + 3] = t.w;
         }
     float *r_out = reinterpret_cast<float *>(blk + codes_bytes(BITS));
-    fit_quantize_pack<4, BITS>(T, ix, rp, xc, blk, r_out, r_out + DK, true);
+    if (a.impact)
+        fit_quantize_pack_impact<BITS>(T, ix, rp, a.impact + (long long)h * DK, blk, r_out, r_out + DK);
+    else
+        fit_quantize_pack<4, BITS>(T, ix, rp, xc, blk, r_out, r_out + DK, true);
 }
 
 __global__ void __launch_bounds__(256) load_fp32_kernel(const IoArgs a, const float *S)
@@ -156,9 +227,9 @@ __global__ void __launch_bounds__(256) load_fp32_kernel(const IoArgs a, const fl
     const float *Si = S + it * DK * DV;
     const TileIdx<4> ix(threadIdx.x);
     switch (a.head_bits[h]) {
-    case 4: load_fp32_item<4>(a, blk, Si, ix, rp, xc); break;
-    case 6: load_fp32_item<6>(a, blk, Si, ix, rp, xc); break;
-    case 8: load_fp32_item<8>(a, blk, Si, ix, rp, xc); break;
+    case 4: load_fp32_item<4>(a, blk, Si, ix, rp, xc, h); break;
+    case 6: load_fp32_item<6>(a, blk, Si, ix, rp, xc, h); break;
+    case 8: load_fp32_item<8>(a, blk, Si, ix, rp, xc, h); break;
     default: {
         // FP16 pivot head: the state rounded to binary16 (nearest, ties to even)
         __half *dst = reinterpret_cast<__half *>(blk);
@@ -251,6 +322,7 @@ IoArgs io_args(const stepq_pool *p, const int32_t *slot_ids)
     a.H = p->H;
     a.slot_ids = slot_ids;
     a.flag = p->d_flag;
+    a.impact = p->d_impact;
     return a;
 }
 

@@ -28,7 +28,7 @@ EXPORTED = [
     "stepq_pool_load_fp32", "stepq_pool_load_packed", "stepq_pool_dump_fp32",
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
-    "stepq_allocate_bits_pivots",
+    "stepq_allocate_bits_pivots", "stepq_pool_set_impact",
 ]
 
 
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_pool_get_error": [P, ctypes.POINTER(I)],
         "stepq_allocate_bits": [P, P, I, P, I, ctypes.c_double, P],
         "stepq_allocate_bits_pivots": [P, P, I, P, I, ctypes.c_double, I, P],
+        "stepq_pool_set_impact": [P, P],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
@@ -177,6 +178,15 @@ def stepq_decode_step_noalloc(num_slots: int, head_bits, num_key_heads: int, gat
         None if flag_out is None else _dev(flag_out, "flag_out"), _stream(stream)), "stepq_decode_step_noalloc")
 
 
+def stepq_pool_set_impact(pool: int, impact=None):
+    """Row-impact scores [H, d_k] (host array) for the impact-weighted fit, or None."""
+    if impact is None:
+        _check(load_library().stepq_pool_set_impact(pool, None), "stepq_pool_set_impact")
+        return
+    w = np.ascontiguousarray(impact, dtype=np.float32)
+    _check(load_library().stepq_pool_set_impact(pool, w.ctypes.data), "stepq_pool_set_impact")
+
+
 def stepq_pool_get_error(pool: int) -> int:
     f = ctypes.c_int32()
     _check(load_library().stepq_pool_get_error(pool, ctypes.byref(f)), "stepq_pool_get_error")
@@ -251,3 +261,8 @@ class Pool:
 
     def get_error(self) -> int:
         return stepq_pool_get_error(self.handle)
+
+    def set_impact(self, impact=None):
+        if impact is not None and np.shape(impact) != (self.H, 128):
+            raise ValueError("impact must be [H, 128]")
+        stepq_pool_set_impact(self.handle, impact)

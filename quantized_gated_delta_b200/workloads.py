@@ -173,6 +173,13 @@ def _make_workload(config: int, variant: str, batch: int | None) -> Workload:
     raise ValueError("unknown workload %r" % config)
 
 
+def impact_scores(w: Workload, layer: int = 0) -> np.ndarray:
+    """Synthetic row-impact scores [H, d_k] for the impact-weighted fit: positive, spread over
+    about two decades (log-normal, sigma 1.2), seeded by (seed, layer).  The pages calibrate
+    them as expected squared readout weights over WikiText-2 tokens; no model or data here."""
+    return np.exp(_rng(w.seed, layer, 7000).normal(0.0, 1.2, (w.H, w.dk))).astype(np.float32)
+
+
 # --------------------------------------------------------------------------- per-step inputs
 
 def step_inputs(w: Workload, t: int, phase: int = PHASE_RUN, layer: int = 0) -> dict:

@@ -13,6 +13,16 @@ R_ULP = 8                   # row factors r within 8 ulp of the oracle's
 C_ULP = 4                   # column factors c within 4 ulp
 Y_MAX_REL = 1e-4            # per (request, head): max_j |dy_j| / max_j |y_j|
 Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
+# Impact-weighted fit: the column scale c_j is the least-squares scale of the intermediate
+# codes Q0, a quotient of two sums of up to 128 non-negative terms; fp32 sums differ from the
+# oracle's double sums by at most ~(n-1) u, so c within 2e-5 relative.  An intermediate code
+# at a near tie may round one level apart (as any code may), which moves c_j by
+# w r^2 |P| / sum w r^2 Q0^2 -- a few percent in a column that a few rows carry; such columns
+# are counted like code flips and may be at most 1e-3 of the columns.  The codes follow c:
+# +-1 at a rate up to 1e-3.
+C_REL_IMPACT = 2e-5
+C_FAR_RATE_IMPACT = 1e-3
+CODE_FLIP_RATE_IMPACT = 1e-3
 PIVOT_ULP = 1               # FP16 pivot states: binary16 values within 1 ulp ...
 PIVOT_FLIP_RATE = 1e-3      # ... and off by one ulp at most at this rate
 
@@ -101,6 +111,12 @@ def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv
             res["elements"] += d.size
             res["r_ulp"] = max(res["r_ulp"], int(ulp_diff(rg, ro).max()))
             res["c_ulp"] = max(res["c_ulp"], int(ulp_diff(cg, co).max()))
+            nz = co != 0
+            rel = np.abs(cg[nz].astype(np.float64) - co[nz]) / np.abs(co[nz]) if nz.any() else np.zeros(1)
+            res["c_rel"] = max(res.get("c_rel", 0.0), float(rel.max()))
+            res["c_far"] = res.get("c_far", 0) + int(np.sum(rel > C_REL_IMPACT))
+            res["c_cols"] = res.get("c_cols", 0) + int(cg.size)
+            res["zero_c_mismatch"] = res.get("zero_c_mismatch", 0) + int(np.sum((co == 0) != (cg == 0)))
     return res
 
 
@@ -118,3 +134,10 @@ def pivots_ok(res: dict) -> bool:
     if res["pivot_elements"] == 0:
         return True
     return res["pivot_ulp"] <= PIVOT_ULP and res["pivot_flips"] <= max(1, PIVOT_FLIP_RATE * res["pivot_elements"])
+
+
+def impact_scales_ok(res: dict) -> bool:
+    """The impact-fit column-scale bar (see C_REL_IMPACT): c within 2e-5 relative except in at
+    most a 1e-3 share of the compared columns, and zero exactly where the oracle's is zero."""
+    cols = res.get("c_cols", 0)
+    return res.get("zero_c_mismatch", 0) == 0 and res.get("c_far", 0) <= max(1, C_FAR_RATE_IMPACT * cols)

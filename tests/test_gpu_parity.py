@@ -402,3 +402,112 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
     assert worst["r_ulp"] <= PH.R_ULP and worst["c_ulp"] <= PH.C_ULP
     assert worst["y"] <= PH.Y_MAX_REL
     assert rel <= PH.Y_TRAJ_REL_L2
+
+
+# --------------------------------------------------------------------------- impact-weighted fit
+
+def _impact_scores(rng, H):
+    """Synthetic row-impact scores (positive, spread over two decades, as calibration gives)."""
+    return np.exp(rng.normal(0, 1.2, (H, 128))).astype(f32)
+
+
+def test_impact_fit_load_and_step_vs_oracle(S):
+    """Pool with row-impact scores: quantize-in and one decode step (GDN fp32, KDA bf16)
+    against the oracle's impact-weighted fit: r within 8 ulp, c within 2e-5, codes +-1 at a
+    rate <= 1e-3, y as always."""
+    rng = np.random.default_rng(13)
+    bits = [4, 6, 8, 6]
+    n, H = 3, 4
+    omega = _impact_scores(rng, H)
+    st = random_states(rng, n, H)
+    ids = np.array([2, 0, 1], np.int32)
+    op = O.OraclePool(3, bits, H, impact=omega)
+    op.load_fp32(ids, st)
+    gp = S.Pool(3, bits, H, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_F32)
+    gp.set_impact(omega)
+    gp.load_fp32(slots_t(ids), dev(st))
+    res = PH.compare_slots(dump_bytes(gp, ids), op.slot_bytes(ids), bits)
+    assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP
+    assert PH.impact_scales_ok(res), res
+    assert res["flips"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"])
+    for gate, dtype, Hk in ((0, S.STEPQ_DTYPE_F32, H), (1, S.STEPQ_DTYPE_BF16, 2)):
+        op2 = O.OraclePool(3, bits, Hk, gate, impact=omega)
+        op2.load_fp32(ids, st)
+        x = dict(q=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)])),
+                 k=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)])),
+                 v=W.round_bf16(rng.standard_normal((n, H, 128)).astype(f32)),
+                 alpha=W.round_bf16(rng.uniform(0.6, 1, (n, H) if gate == 0 else (n, H, 128)).astype(f32)),
+                 beta=W.round_bf16(rng.uniform(0.1, 0.9, (n, H)).astype(f32)))
+        gp2 = S.Pool(3, bits, Hk, gate, dtype)
+        gp2.set_impact(omega)
+        load_bytes(gp2, ids, op2.slot_bytes(ids))
+        tx = {}
+        for key, val in x.items():
+            tx[key] = dev(W.to_bf16_bits(val).view(np.int16)) if dtype == S.STEPQ_DTYPE_BF16 else dev(val)
+        y = torch.empty((n, H, 128), device="cuda")
+        gp2.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        yo = op2.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+        assert gp2.get_error() == 0
+        res = PH.compare_slots(dump_bytes(gp2, ids), op2.slot_bytes(ids), bits)
+        assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP, res
+        assert PH.impact_scales_ok(res), res
+        assert res["flips"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"]), res
+        assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL
+
+
+def test_impact_fit_trajectory_config4(S):
+    """Config-4 pool with synthetic row-impact scores, full batch on the GPU, a sampled
+    trajectory on the oracle (re-synchronised after a code difference, as for the clip-free
+    fit); unit scores select the impact fit too, and clearing them returns to the clip-free fit."""
+    w = W.make_workload(4, "mixed6")
+    bits = PH.head_bits(w)
+    rng = np.random.default_rng(14)
+    omega = _impact_scores(rng, w.H)
+    sub = W.sample_requests(w, 4)
+    sub_slots = w.slot_ids[sub]
+    op = PH.oracle_pool_with_warmup(w, bits, sub)
+    op_imp = O.OraclePool(w.num_slots, bits, w.Hk, w.gate_mode, impact=omega)
+    op_imp.data[:] = op.data
+    gp = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    gp.set_impact(omega)
+    load_bytes(gp, sub_slots, op_imp.slot_bytes(sub_slots))
+    all_slots = slots_t(w.slot_ids)
+    flips = elements = c_far = c_cols = 0
+    worst = dict(r_ulp=0, c_rel=0.0, y=0.0)
+    for t in range(24):
+        x = W.step_inputs(w, t)
+        tx = PH.to_device(w, x, torch)
+        y = torch.empty((w.B, w.H, w.dv), device="cuda")
+        gp.decode_step(all_slots, tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        xs = PH.sub_inputs(x, sub)
+        yo = op_imp.decode_step(sub_slots, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"])
+        yg = y[torch.from_numpy(sub).cuda()].cpu().numpy()
+        worst["y"] = max(worst["y"], PH.y_max_rel(yg, yo))
+        gb, ob = dump_bytes(gp, sub_slots), op_imp.slot_bytes(sub_slots)
+        res = PH.compare_slots(gb, ob, bits)
+        assert res["max_code_diff"] <= 1 and res.get("zero_c_mismatch", 0) == 0
+        flips += res["flips"]
+        elements += res["elements"]
+        c_far += res.get("c_far", 0)
+        c_cols += res.get("c_cols", 0)
+        worst["r_ulp"] = max(worst["r_ulp"], res["r_ulp"])
+        worst["c_rel"] = max(worst["c_rel"], res.get("c_rel", 0.0))
+        if not res["byte_equal"]:
+            load_bytes(gp, sub_slots, ob)
+    print("\nimpact fit: worst %s, flips %d / %d (%.2e), columns with c off > 2e-5: %d / %d" %
+          (worst, flips, elements, flips / elements, c_far, c_cols))
+    assert gp.get_error() == 0
+    assert worst["r_ulp"] <= PH.R_ULP and worst["y"] <= PH.Y_MAX_REL
+    assert c_far <= max(1, PH.C_FAR_RATE_IMPACT * c_cols)
+    assert flips <= PH.CODE_FLIP_RATE_IMPACT * elements
+    # clearing the scores returns to the clip-free fit
+    gp.set_impact(None)
+    load_bytes(gp, sub_slots, op.slot_bytes(sub_slots))
+    x = W.step_inputs(w, 0)
+    tx = PH.to_device(w, x, torch)
+    y = torch.empty((w.B, w.H, w.dv), device="cuda")
+    gp.decode_step(all_slots, tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    xs = PH.sub_inputs(x, sub)
+    op.decode_step(sub_slots, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"])
+    res = PH.compare_slots(dump_bytes(gp, sub_slots), op.slot_bytes(sub_slots), bits)
+    assert res["max_code_diff"] <= 1 and res["c_ulp"] <= PH.C_ULP
