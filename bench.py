@@ -40,8 +40,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=4096)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="mixed6", choices=["mixed6", "uniform4", "mixed6p"],
-                    help="mixed6: 6-bit nominal allocation; uniform4; mixed6p: mixed6 plus one FP16 pivot head")
+    ap.add_argument("--variant", default="mixed6", choices=["mixed6", "uniform4", "mixed6p", "rowbits"],
+                    help="mixed6: 6-bit nominal allocation; uniform4; mixed6p: mixed6 plus one FP16 pivot head; "
+                         "rowbits (--workload kda): per-key-row widths")
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -49,8 +50,9 @@ def parse():
                     help="distinct per-step input batches kept on the device and cycled")
     ap.add_argument("--fit", default="clipfree", choices=["clipfree", "impact"],
                     help="dual-axis fit: clip-free (the headline) or impact-weighted with synthetic row-impact scores")
-    ap.add_argument("--workload", default="pool", choices=["pool", "stack"],
-                    help="pool: the high-concurrency pool (the headline); stack: the 36-layer stack sweep")
+    ap.add_argument("--workload", default="pool", choices=["pool", "stack", "kda"],
+                    help="pool: the high-concurrency pool (the headline); stack: the 36-layer stack sweep; "
+                         "kda: the KDA layer (per-channel gates)")
     ap.add_argument("--batch", type=int, default=1024, choices=[64, 256, 1024],
                     help="requests of the stack sweep")
     return ap.parse_args()
@@ -148,9 +150,11 @@ def block_bytes(bits: int, dk: int = 128, dv: int = 128) -> int:
     return dk * dv * bits // 8 + 4 * dk + 4 * dv
 
 
-def algorithmic_bytes_per_step(w, bits) -> float:
-    """State read once + written once per (request, head), plus the step's inputs and outputs."""
-    state = 2.0 * w.B * sum(block_bytes(int(b), w.dk, w.dv) for b in bits)
+def algorithmic_bytes_per_step(w, bits, slot_stride=None) -> float:
+    """State read once + written once per (request, head), plus the step's inputs and outputs
+    (slot_stride: the pool's bytes per request, for heads with per-key-row widths)."""
+    per_slot = slot_stride if slot_stride is not None else sum(block_bytes(int(b), w.dk, w.dv) for b in bits)
+    state = 2.0 * w.B * per_slot
     esz = 2 if w.in_dtype == 1 else 4
     io = w.B * w.Hk * 2 * w.dk * esz            # q, k (shared by H / Hk value heads)
     io += w.B * w.H * w.dv * esz                # v
@@ -336,16 +340,22 @@ def main():
     torch.cuda.set_device(local)
     rank, world, local = D.init_from_env("nccl", timeout_s=120)
 
-    w = W.make_workload(4, args.variant)
+    w = W.make_workload(3 if args.workload == "kda" else 4, args.variant)
     w.seed = D.shard_seed(w.seed, rank)              # each rank serves its own requests
-    if w.head_bits is not None:
+    row_bits = None
+    if w.row_half_life is not None:
+        # the allocation unit is the key row: widths over the layer's H * d_k rows
+        rb = stepq.stepq_allocate_bits(np.ravel(w.row_half_life[0]), None, (4, 6, 8), w.avg_bits)
+        row_bits = np.asarray(rb, np.uint8).reshape(w.H, w.dk)
+        bits = np.zeros(w.H, dtype=np.uint8)
+    elif w.head_bits is not None:
         bits = w.head_bits[0]
     elif w.n_pivots:
         bits = stepq.stepq_allocate_bits_pivots(w.half_life[0], None, (4, 6, 8), w.avg_bits, w.n_pivots)
     else:
         bits = stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits)
     bits = np.asarray(bits, dtype=np.uint8)
-    pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype, row_bits=row_bits)
     if args.fit == "impact":
         pool.set_impact(W.impact_scores(w))
     slots = torch.from_numpy(w.slot_ids).cuda()
@@ -395,7 +405,7 @@ def main():
     units_per_step = w.B * w.H
     value = units_per_step * args.steps * world / (ms_total / 1e3)
     avg_kernel_s = (sum(kernel_ms) / len(kernel_ms)) / 1e3
-    alg_bytes = algorithmic_bytes_per_step(w, bits)
+    alg_bytes = algorithmic_bytes_per_step(w, bits, pool.slot_stride)
     peak, peak_kind = peaks()
     achieved = alg_bytes / avg_kernel_s / 1e9
 
@@ -431,7 +441,7 @@ def main():
     e2e_value = units_per_step * args.e2e_steps * world / (ms_e2e / 1e3)
 
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and row_bits is None:
         base = cpu_baseline(w, bits, args.cpu_seconds)
 
     if rank == 0:
@@ -441,11 +451,13 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s%s"
                        % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
-                          "".join(str(int(b)) for b in bits),
+                          "".join(str(int(b)) for b in bits) if row_bits is None else "per key row (4/6/8: %s)"
+                          % "/".join(str(int(np.sum(row_bits == x))) for x in (4, 6, 8)),
                           ", impact-weighted fit" if args.fit == "impact" else ""),
-                       "avg_bits": float(np.mean(bits)), "parallelism": "dp%d (independent pools)" % world,
+                       "avg_bits": float(np.mean(bits if row_bits is None else row_bits)),
+                       "parallelism": "dp%d (independent pools)" % world,
                        "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
-                             % (w.B * sum(block_bytes(int(b)) for b in bits) / 1e6),
+                             % (w.B * pool.slot_stride / 1e6),
                        "input_sets": nsets},
             "achieved_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -98,6 +98,19 @@ typedef struct {
  * head_bits are copied.  Synchronizes the device.  [BLOG: pool with spare slots] */
 STEPQ_API int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out);
 
+/* Pool whose heads of width 0 carry per-key-row widths.      [BLOG: the allocation unit of
+ * Kimi's KDA is a single key row]  desc as for stepq_pool_create, except that head_bits[h]
+ * may be 0; row_bits (HOST [H, d_k], entries in {4, 6, 8}) then gives the width of each key
+ * row of head h (entries of other heads are ignored).  Such a head stores its rows grouped
+ * by width -- 8-bit rows, then 4-bit, then 6-bit, each group in ascending key-row order --
+ * with each 16-column panel holding one segment of 16 codes per stored row at the row's
+ * width, padded to a multiple of 16 bytes; then r[d_k] in stored-row order, then c[d_v].
+ * Block bytes = 8 * roundup16(16 n8 + 8 n4 + 12 n6) + 4 d_k + 4 d_v.  The fit is the clip-free
+ * fit at each row's own levels (qmax = 2^(b_i - 1) - 1); the impact-weighted fit
+ * (stepq_pool_set_impact) applies to the heads of uniform width only.  The allocation-free
+ * entry point does not take such pools. */
+STEPQ_API int stepq_pool_create_rows(const stepq_pool_desc *desc, const uint8_t *row_bits, stepq_pool **out);
+
 /* Free the pool and its device memory.  Synchronizes the device.  NULL is a no-op. */
 STEPQ_API int stepq_pool_destroy(stepq_pool *pool);
 

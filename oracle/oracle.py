@@ -60,12 +60,18 @@ def _load():
         "oracle_dequantize": (None, [I, I, P, P, P, P]),
         "oracle_delta_step": (None, [I, I, P, P, P, P, P, F, P]),
         "oracle_step_state": (I, [I, I, I, P, P, P, P, P, P, P, F, P, P, P, P, P]),
-        "oracle_head_offsets": (L, [I, P, I, I, P]),
-        "oracle_decode_step": (L, [I, I, I, I, I, P, I, P, P, I, P, P, P, P, P, P, I, P]),
-        "oracle_pool_load": (L, [I, I, I, P, I, P, P, I, P, I, P]),
+        "oracle_head_offsets": (L, [I, P, I, I, P, P]),
+        "oracle_decode_step": (L, [I, I, I, I, I, P, I, P, P, I, P, P, P, P, P, P, I, P, P]),
+        "oracle_pool_load": (L, [I, I, I, P, I, P, P, I, P, I, P, P]),
         "oracle_impact_normalize": (None, [I, P, P]),
         "oracle_quantize_impact": (I, [I, I, I, P, P, P, P, P]),
-        "oracle_pool_dump": (I, [I, I, I, P, I, P, P, I, P, I]),
+        "oracle_pool_dump": (I, [I, I, I, P, I, P, P, I, P, I, P]),
+        "oracle_rows_order": (None, [I, P, P]),
+        "oracle_rows_panel_bytes": (L, [I, P]),
+        "oracle_rows_block_bytes": (L, [I, I, P]),
+        "oracle_rows_pack": (None, [I, I, P, P, P]),
+        "oracle_rows_unpack": (None, [I, I, P, P, P]),
+        "oracle_rows_quantize": (I, [I, I, P, P, P, P, P]),
         "oracle_fp_decode_step": (None, [I, I, I, I, I, I, P, P, P, P, P, P, P, I, I]),
         "oracle_fp16_encode": (None, [L, P, P]),
         "oracle_fp16_decode": (None, [L, P, P]),
@@ -104,12 +110,71 @@ def block_bytes(bits: int, dk: int = 128, dv: int = 128) -> int:
     return _load().oracle_block_bytes(bits, dk, dv)
 
 
-def head_offsets(head_bits, dk: int = 128, dv: int = 128):
-    """(offsets[H], slot_stride) of the head blocks inside one slot."""
+def head_offsets(head_bits, dk: int = 128, dv: int = 128, row_bits=None):
+    """(offsets[H], slot_stride) of the head blocks inside one slot (a head of width 0 takes
+    its per-key-row widths from row_bits [H, dk])."""
     hb = _c(head_bits, np.int32)
     off = np.zeros(len(hb), dtype=np.int64)
-    stride = _load().oracle_head_offsets(len(hb), _p(hb), dk, dv, _p(off))
+    rb = None if row_bits is None else _c(row_bits, np.int32)
+    stride = _load().oracle_head_offsets(len(hb), _p(hb), dk, dv, _p(off), None if rb is None else _p(rb))
     return off, int(stride)
+
+
+# --------------------------------------------------------------------------- per-key-row widths
+
+def rows_order(rb) -> np.ndarray:
+    """Stored position -> key row of a head with per-row widths rb [dk]."""
+    rb = _c(rb, np.int32)
+    out = np.zeros(len(rb), dtype=np.int32)
+    _load().oracle_rows_order(len(rb), _p(rb), _p(out))
+    return out
+
+
+def rows_block_bytes(rb, dv: int = 128) -> int:
+    rb = _c(rb, np.int32)
+    return int(_load().oracle_rows_block_bytes(len(rb), dv, _p(rb)))
+
+
+def rows_pack(Q: np.ndarray, rb) -> np.ndarray:
+    Q = _c(Q, np.int32)
+    rb = _c(rb, np.int32)
+    dk, dv = Q.shape
+    out = np.zeros(rows_block_bytes(rb, dv) - 4 * dk - 4 * dv, dtype=np.uint8)
+    _load().oracle_rows_pack(dk, dv, _p(rb), _p(Q), _p(out))
+    return out
+
+
+def rows_unpack(buf: np.ndarray, rb, dv: int = 128) -> np.ndarray:
+    buf = _c(buf, np.uint8)
+    rb = _c(rb, np.int32)
+    Q = np.zeros((len(rb), dv), dtype=np.int32)
+    _load().oracle_rows_unpack(len(rb), dv, _p(rb), _p(buf), _p(Q))
+    return Q
+
+
+def rows_split_block(blk: np.ndarray, rb, dv: int = 128):
+    """Per-row head block -> (Q [dk, dv], r [dk] by key row, c [dv])."""
+    rb = _c(rb, np.int32)
+    dk = len(rb)
+    blk = _c(blk, np.uint8)
+    cb = rows_block_bytes(rb, dv) - 4 * dk - 4 * dv
+    Q = rows_unpack(blk[:cb], rb, dv)
+    r = np.zeros(dk, dtype=np.float32)
+    r[rows_order(rb)] = blk[cb:cb + 4 * dk].view(np.float32)
+    c = blk[cb + 4 * dk:cb + 4 * dk + 4 * dv].view(np.float32).copy()
+    return Q, r, c
+
+
+def rows_quantize(S32: np.ndarray, rb):
+    """Clip-free fit at each row's own levels -> (Q, r, c, clipped)."""
+    S32 = _c(S32, np.float32)
+    rb = _c(rb, np.int32)
+    dk, dv = S32.shape
+    Q = np.zeros((dk, dv), dtype=np.int32)
+    r = np.zeros(dk, dtype=np.float32)
+    c = np.zeros(dv, dtype=np.float32)
+    n = _load().oracle_rows_quantize(dk, dv, _p(rb), _p(S32), _p(Q), _p(r), _p(c))
+    return Q, r, c, int(n)
 
 
 def pack_codes(Q: np.ndarray, bits: int) -> np.ndarray:
@@ -250,7 +315,7 @@ class OraclePool:
     binary16 values).  A zeroed pool is the zero state."""
 
     def __init__(self, num_slots: int, head_bits, num_key_heads: int, gate_mode: int = 0,
-                 dk: int = 128, dv: int = 128, impact=None):
+                 dk: int = 128, dv: int = 128, impact=None, row_bits=None):
         self.head_bits = _c(head_bits, np.int32)
         self.H = len(self.head_bits)
         self.Hk = int(num_key_heads)
@@ -259,7 +324,10 @@ class OraclePool:
         self.dk, self.dv = dk, dv
         self.gate_mode = int(gate_mode)
         self.num_slots = int(num_slots)
-        self.offsets, self.slot_stride = head_offsets(self.head_bits, dk, dv)
+        self.row_bits = None if row_bits is None else _c(row_bits, np.int32)
+        if (self.head_bits == 0).any():
+            assert self.row_bits is not None and self.row_bits.shape == (self.H, dk)
+        self.offsets, self.slot_stride = head_offsets(self.head_bits, dk, dv, self.row_bits)
         self.data = np.zeros(self.num_slots * self.slot_stride, dtype=np.uint8)
         # row-impact scores [H, dk] -> the impact-weighted fit for every quantized head
         self.impact_w = None
@@ -268,18 +336,27 @@ class OraclePool:
             assert impact.shape == (self.H, dk) and (impact > 0).all()
             self.impact_w = np.stack([impact_normalize(row) for row in impact])
 
+    def block_size(self, h: int) -> int:
+        b = int(self.head_bits[h])
+        return block_bytes(b, self.dk, self.dv) if b else rows_block_bytes(self.row_bits[h], self.dv)
+
     def block(self, slot: int, h: int) -> np.ndarray:
         o = slot * self.slot_stride + int(self.offsets[h])
-        return self.data[o:o + block_bytes(int(self.head_bits[h]), self.dk, self.dv)]
+        return self.data[o:o + self.block_size(h)]
 
     def state(self, slot: int, h: int):
         """(Q, r, c) of a quantized head; the binary16 bit patterns of an FP16 pivot head."""
         if int(self.head_bits[h]) == 16:
             return pivot_state(self.block(slot, h), self.dk, self.dv)
+        if int(self.head_bits[h]) == 0:
+            return rows_split_block(self.block(slot, h), self.row_bits[h], self.dv)
         return split_block(self.block(slot, h), int(self.head_bits[h]), self.dk, self.dv)
 
     def set_state(self, slot: int, h: int, Q, r, c):
         self.block(slot, h)[:] = make_block(Q, r, c, int(self.head_bits[h]))
+
+    def _rb(self):
+        return None if self.row_bits is None else _p(self.row_bits)
 
     def slot_bytes(self, slot_ids) -> np.ndarray:
         s = self.slot_stride
@@ -292,7 +369,7 @@ class OraclePool:
         assert S.shape == (len(sl), self.H, self.dk, self.dv)
         rc = _load().oracle_pool_load(self.H, self.dk, self.dv, _p(self.head_bits), self.num_slots,
                                       _p(self.data), _p(sl), len(sl), _p(S), nthreads or default_threads(),
-                                      None if self.impact_w is None else _p(self.impact_w))
+                                      None if self.impact_w is None else _p(self.impact_w), self._rb())
         if rc < 0:
             raise IndexError("slot id out of range")
         return int(rc)
@@ -301,7 +378,8 @@ class OraclePool:
         sl = _c(slot_ids, np.int32)
         S = np.zeros((len(sl), self.H, self.dk, self.dv), dtype=np.float32)
         rc = _load().oracle_pool_dump(self.H, self.dk, self.dv, _p(self.head_bits), self.num_slots,
-                                      _p(self.data), _p(sl), len(sl), _p(S), nthreads or default_threads())
+                                      _p(self.data), _p(sl), len(sl), _p(S), nthreads or default_threads(),
+                                      self._rb())
         if rc < 0:
             raise IndexError("slot id out of range")
         return S
@@ -323,7 +401,7 @@ class OraclePool:
                                         _p(self.head_bits), self.num_slots, _p(self.data), _p(sl), n,
                                         _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(y),
                                         nthreads or default_threads(),
-                                        None if self.impact_w is None else _p(self.impact_w))
+                                        None if self.impact_w is None else _p(self.impact_w), self._rb())
         if rc < 0:
             raise IndexError("slot id out of range")
         if rc > 0:
@@ -405,6 +483,40 @@ def allocate_bits_pivots(half_life, distortion, cand, avg_bits, n_pivots: int):
     for u, b in zip(rest, bits_rest):
         bits[u] = b
     return bits, obj
+
+
+def allocate_bits_dp_vec(half_life, distortion, cand, avg_bits):
+    """The same exact programme vectorised over the bits spent (numpy), for thousands of
+    units (one unit per key row).  Ties resolve as in the library's allocator: for each total
+    the widest candidate that reaches the best value first, then the smallest total."""
+    N = len(half_life)
+    budget = math.floor(N * avg_bits + 1e-9)
+    cand = list(cand)
+    order = sorted(range(len(cand)), key=lambda ci: -cand[ci])          # widest first
+    best = np.full(budget + 1, np.inf)
+    best[0] = 0.0
+    choice = np.full((N, budget + 1), -1, dtype=np.int8)
+    for u in range(N):
+        w = -1.0 / math.expm1(-math.log(2.0) / half_life[u])
+        nxt = np.full(budget + 1, np.inf)
+        pick = np.full(budget + 1, -1, dtype=np.int8)
+        for ci in order:
+            b = cand[ci]
+            v = np.full(budget + 1, np.inf)
+            v[b:] = best[:budget + 1 - b] + w * _distortion(distortion, u, ci, cand)
+            better = v < nxt
+            nxt = np.where(better, v, nxt)
+            pick = np.where(better, ci, pick)
+        best, choice[u] = nxt, pick
+    if not np.isfinite(best).any():
+        raise ValueError("budget too small for the candidate widths")
+    s = int(np.argmin(best))
+    bits = [0] * N
+    for u in range(N - 1, -1, -1):
+        ci = int(choice[u, s])
+        bits[u] = cand[ci]
+        s -= cand[ci]
+    return bits, float(np.min(best))
 
 
 def allocate_bits_dp(half_life, distortion, cand, avg_bits):

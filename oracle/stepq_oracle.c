@@ -159,6 +159,87 @@ void oracle_unpack_codes(int bits, int dk, int dv, const uint8_t *in, int32_t *Q
 }
 
 /* ------------------------------------------------------------------------- */
+/* Per-key-row widths ([BLOG]: the allocation unit of Kimi's KDA is a single key */
+/* row)                                                                        */
+/* ------------------------------------------------------------------------- */
+/* A head whose key rows carry their own widths rb[i] in {4, 6, 8}.  Readings (the pages
+ * give no layout): the rows are stored grouped by width -- 8-bit rows, then 4-bit, then
+ * 6-bit, each group in ascending key-row order -- so each width's segments stay aligned;
+ * a panel (16 value columns) holds one segment of 16 codes per stored row (the row's
+ * width, a little-endian bit stream of offset-binary fields), padded to a multiple of 16
+ * bytes; the head block is the 8 panels, then r[d_k] in stored-row order, then c[d_v].
+ * With every rb[i] = b this is exactly the uniform layout above. */
+
+/* Stored position -> key row. */
+void oracle_rows_order(int dk, const int32_t *rb, int32_t *order)
+{
+    const int widths[3] = {8, 4, 6};
+    int p = 0;
+    for (int w = 0; w < 3; w++)
+        for (int i = 0; i < dk; i++)
+            if (rb[i] == widths[w]) order[p++] = i;
+}
+
+long oracle_rows_panel_bytes(int dk, const int32_t *rb)
+{
+    long sum = 0;
+    for (int i = 0; i < dk; i++) sum += 2L * rb[i];              /* 16 codes of rb[i] bits */
+    return (sum + 15) / 16 * 16;
+}
+
+long oracle_rows_block_bytes(int dk, int dv, const int32_t *rb)
+{
+    return (long)(dv / ORACLE_PANEL) * oracle_rows_panel_bytes(dk, rb) + 4L * dk + 4L * dv;
+}
+
+/* Codes Q[dk*dv] (key-row-major) of a per-row head into its code region; one bit at a time. */
+void oracle_rows_pack(int dk, int dv, const int32_t *rb, const int32_t *Q, uint8_t *out)
+{
+    int32_t *order = (int32_t *)malloc((size_t)dk * sizeof(int32_t));
+    oracle_rows_order(dk, rb, order);
+    const long panel = oracle_rows_panel_bytes(dk, rb);
+    memset(out, 0, (size_t)((dv / ORACLE_PANEL) * panel));
+    for (int pj = 0; pj < dv / ORACLE_PANEL; pj++) {
+        long seg = pj * panel;                                   /* byte offset of the segment */
+        for (int p = 0; p < dk; p++) {
+            const int i = order[p], b = rb[i];
+            for (int jj = 0; jj < ORACLE_PANEL; jj++) {
+                uint32_t u = (uint32_t)(Q[(long)i * dv + pj * ORACLE_PANEL + jj] + (1 << (b - 1)));
+                for (int t = 0; t < b; t++) {
+                    long bit = seg * 8 + (long)jj * b + t;
+                    if ((u >> t) & 1u) out[bit / 8] |= (uint8_t)(1u << (bit % 8));
+                }
+            }
+            seg += 2L * b;
+        }
+    }
+    free(order);
+}
+
+void oracle_rows_unpack(int dk, int dv, const int32_t *rb, const uint8_t *in, int32_t *Q)
+{
+    int32_t *order = (int32_t *)malloc((size_t)dk * sizeof(int32_t));
+    oracle_rows_order(dk, rb, order);
+    const long panel = oracle_rows_panel_bytes(dk, rb);
+    for (int pj = 0; pj < dv / ORACLE_PANEL; pj++) {
+        long seg = pj * panel;
+        for (int p = 0; p < dk; p++) {
+            const int i = order[p], b = rb[i];
+            for (int jj = 0; jj < ORACLE_PANEL; jj++) {
+                uint32_t u = 0;
+                for (int t = 0; t < b; t++) {
+                    long bit = seg * 8 + (long)jj * b + t;
+                    u |= (uint32_t)((in[bit / 8] >> (bit % 8)) & 1u) << t;
+                }
+                Q[(long)i * dv + pj * ORACLE_PANEL + jj] = (int32_t)u - (1 << (b - 1));
+            }
+            seg += 2L * b;
+        }
+    }
+    free(order);
+}
+
+/* ------------------------------------------------------------------------- */
 /* Quantization: dual-axis fit + nearest level ([SUM] Method para 4)          */
 /* ------------------------------------------------------------------------- */
 
@@ -198,6 +279,40 @@ int oracle_quantize(int bits, int dk, int dv, const float *S32, int32_t *Q, floa
             if (qv < -qmax) { qv = -qmax; clipped++; }
             Q[(long)i * dv + j] = (int32_t)qv;
         }
+    return clipped;
+}
+
+/* The clip-free fit with each key row's own width: c_j = sqrt(max_i |S_ij|),
+ * r_i = max_j (|S_ij| / c_j) / qmax(rb[i]), codes at the row's levels. */
+int oracle_rows_quantize(int dk, int dv, const int32_t *rb, const float *S32, int32_t *Q, float *r, float *c)
+{
+    int clipped = 0;
+    for (int j = 0; j < dv; j++) {
+        double M = 0.0;
+        for (int i = 0; i < dk; i++) {
+            double a = fabs((double)S32[(long)i * dv + j]);
+            if (a > M) M = a;
+        }
+        c[j] = (float)sqrt(M);
+    }
+    for (int i = 0; i < dk; i++) {
+        const int qmax = oracle_qmax(rb[i]);
+        double m = 0.0;
+        for (int j = 0; j < dv; j++)
+            if (c[j] > 0.0f) {
+                double t = fabs((double)S32[(long)i * dv + j]) / (double)c[j];
+                if (t > m) m = t;
+            }
+        r[i] = (float)(m / (double)qmax);
+        for (int j = 0; j < dv; j++) {
+            double scale = (double)r[i] * (double)c[j];
+            double x = scale > 0.0 ? (double)S32[(long)i * dv + j] / scale : 0.0;
+            double qv = nearbyint(x);
+            if (qv > qmax) { qv = qmax; clipped++; }
+            if (qv < -qmax) { qv = -qmax; clipped++; }
+            Q[(long)i * dv + j] = (int32_t)qv;
+        }
+    }
     return clipped;
 }
 
@@ -343,6 +458,25 @@ int oracle_step_state_impact(int dk, int dv, int bits, const int32_t *Q_in, cons
                           NULL, w);
 }
 
+/* The same step for a head with per-key-row widths rb[dk]: the clip-free fit at each row's
+ * levels.  Returns the clip count (0 when the fit holds). */
+int oracle_step_state_rows(int dk, int dv, const int32_t *rb, const int32_t *Q_in, const float *r_in,
+                           const float *c_in, const float *q, const float *k, const float *v, const float *alpha,
+                           float beta, int32_t *Q_out, float *r_out, float *c_out, float *y_out)
+{
+    long ne = (long)dk * dv;
+    double *S = (double *)malloc((size_t)ne * sizeof(double));
+    double *y = (double *)malloc((size_t)dv * sizeof(double));
+    float *S32 = (float *)malloc((size_t)ne * sizeof(float));
+    oracle_dequantize(dk, dv, Q_in, r_in, c_in, S);
+    oracle_delta_step(dk, dv, S, q, k, v, alpha, beta, y);
+    for (int j = 0; j < dv; j++) y_out[j] = (float)y[j];
+    for (long e = 0; e < ne; e++) S32[e] = (float)S[e];
+    int clipped = oracle_rows_quantize(dk, dv, rb, S32, Q_out, r_out, c_out);
+    free(S); free(y); free(S32);
+    return clipped;
+}
+
 static int step_state_fit(int dk, int dv, int bits, const int32_t *Q_in, const float *r_in, const float *c_in,
                           const float *q, const float *k, const float *v, const float *alpha, float beta,
                           int32_t *Q_out, float *r_out, float *c_out, float *y_out, double *S_pre,
@@ -367,28 +501,53 @@ static int step_state_fit(int dk, int dv, int bits, const int32_t *Q_in, const f
 /* Pool-level drivers (slot-major pool of packed head blocks)                 */
 /* ------------------------------------------------------------------------- */
 
-/* Byte offset of each head block inside a slot, and the slot stride. */
-long oracle_head_offsets(int H, const int32_t *head_bits, int dk, int dv, long *offsets)
+/* Byte offset of each head block inside a slot, and the slot stride.  A head of width 0
+ * has per-key-row widths row_bits[h * dk .. h * dk + dk) (row_bits may be NULL otherwise). */
+long oracle_head_offsets(int H, const int32_t *head_bits, int dk, int dv, long *offsets, const int32_t *row_bits)
 {
     long off = 0;
     for (int h = 0; h < H; h++) {
         offsets[h] = off;
-        off += oracle_block_bytes(head_bits[h], dk, dv);
+        off += head_bits[h] ? oracle_block_bytes(head_bits[h], dk, dv)
+                            : oracle_rows_block_bytes(dk, dv, row_bits + (long)h * dk);
     }
     return off;
 }
 
-/* Read one head block into codes + scales. */
-static void read_block(const uint8_t *blk, int bits, int dk, int dv, int32_t *Q, float *r, float *c)
+/* Read one head block into codes + scales (r by key row).  rb: the per-row widths of a
+ * head of width 0, else NULL. */
+static void read_block(const uint8_t *blk, int bits, const int32_t *rb, int dk, int dv, int32_t *Q, float *r,
+                       float *c)
 {
+    if (rb) {
+        const long cb = (long)(dv / ORACLE_PANEL) * oracle_rows_panel_bytes(dk, rb);
+        int32_t *order = (int32_t *)malloc((size_t)dk * sizeof(int32_t));
+        oracle_rows_order(dk, rb, order);
+        oracle_rows_unpack(dk, dv, rb, blk, Q);
+        for (int p = 0; p < dk; p++) memcpy(&r[order[p]], blk + cb + 4L * p, 4);
+        memcpy(c, blk + cb + 4L * dk, 4L * dv);
+        free(order);
+        return;
+    }
     long cb = oracle_codes_bytes(bits, dk, dv);
     oracle_unpack_codes(bits, dk, dv, blk, Q);
     memcpy(r, blk + cb, 4L * dk);
     memcpy(c, blk + cb + 4L * dk, 4L * dv);
 }
 
-static void write_block(uint8_t *blk, int bits, int dk, int dv, const int32_t *Q, const float *r, const float *c)
+static void write_block(uint8_t *blk, int bits, const int32_t *rb, int dk, int dv, const int32_t *Q, const float *r,
+                        const float *c)
 {
+    if (rb) {
+        const long cb = (long)(dv / ORACLE_PANEL) * oracle_rows_panel_bytes(dk, rb);
+        int32_t *order = (int32_t *)malloc((size_t)dk * sizeof(int32_t));
+        oracle_rows_order(dk, rb, order);
+        oracle_rows_pack(dk, dv, rb, Q, blk);
+        for (int p = 0; p < dk; p++) memcpy(blk + cb + 4L * p, &r[order[p]], 4);
+        memcpy(blk + cb + 4L * dk, c, 4L * dv);
+        free(order);
+        return;
+    }
     long cb = oracle_codes_bytes(bits, dk, dv);
     oracle_pack_codes(bits, dk, dv, Q, blk);
     memcpy(blk + cb, r, 4L * dk);
@@ -401,16 +560,19 @@ static void write_block(uint8_t *blk, int bits, int dk, int dv, const int32_t *Q
  *   q, k      [n, Hk, dk]; v [n, H, dv]; beta [n, H]
  *   alpha     gate_mode 0 (GDN): [n, H];  gate_mode 1 (KDA): [n, H, dk]
  *   y         [n, H, dv] (fp32 out)
- *   impact    NULL (clip-free fit) or [H, dk] normalized row-impact weights (impact fit)
+ *   impact    NULL (clip-free fit) or [H, dk] normalized row-impact weights (impact fit of
+ *             the uniform-width heads)
+ *   row_bits  [H, dk] per-key-row widths of the heads of width 0 (NULL if there are none)
  * Value head h reads key head h / (H / Hk).  Returns the clip count of the clip-free fit
  * (0 when it holds), or -1 for an out-of-range slot id (that request is skipped). */
 long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int32_t *head_bits,
                         int num_slots, uint8_t *pool, const int32_t *slot_ids, int n,
                         const float *q, const float *k, const float *v, const float *alpha,
-                        const float *beta, float *y, int nthreads, const float *impact)
+                        const float *beta, float *y, int nthreads, const float *impact,
+                        const int32_t *row_bits)
 {
     long *offsets = (long *)malloc((size_t)H * sizeof(long));
-    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets, row_bits);
     long clipped = 0;
     int bad = 0;
     int group = H / Hk;
@@ -444,10 +606,15 @@ long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int3
         float *r2 = (float *)malloc(4L * dk), *c2 = (float *)malloc(4L * dv);
         float *al = (float *)malloc(4L * dk);
         uint8_t *blk = pool + (long)slot * stride + offsets[h];
-        read_block(blk, bits, dk, dv, Q, r, c);
+        const int32_t *rb = bits ? NULL : row_bits + (long)h * dk;
+        read_block(blk, bits, rb, dk, dv, Q, r, c);
         for (int i = 0; i < dk; i++)
             al[i] = gate_mode == 0 ? alpha[(long)b * H + h] : alpha[((long)b * H + h) * dk + i];
-        if (impact)
+        if (rb)
+            clipped += oracle_step_state_rows(dk, dv, rb, Q, r, c, q + ((long)b * Hk + g) * dk,
+                                              k + ((long)b * Hk + g) * dk, v + ((long)b * H + h) * dv, al,
+                                              beta[(long)b * H + h], Q2, r2, c2, y + ((long)b * H + h) * dv);
+        else if (impact)
             (void)oracle_step_state_impact(dk, dv, bits, Q, r, c, q + ((long)b * Hk + g) * dk,
                                            k + ((long)b * Hk + g) * dk, v + ((long)b * H + h) * dv, al,
                                            beta[(long)b * H + h], impact + (long)h * dk, Q2, r2, c2,
@@ -457,20 +624,21 @@ long oracle_decode_step(int H, int Hk, int dk, int dv, int gate_mode, const int3
                                          q + ((long)b * Hk + g) * dk, k + ((long)b * Hk + g) * dk,
                                          v + ((long)b * H + h) * dv, al, beta[(long)b * H + h],
                                          Q2, r2, c2, y + ((long)b * H + h) * dv, NULL);
-        write_block(blk, bits, dk, dv, Q2, r2, c2);
+        write_block(blk, bits, rb, dk, dv, Q2, r2, c2);
         free(Q); free(Q2); free(r); free(c); free(r2); free(c2); free(al);
     }
     free(offsets);
     return bad ? -1 : clipped;
 }
 
-/* Quantize fp32 states S [n, H, dk, dv] into the slots slot_ids[n] of a pool (impact: as for
- * oracle_decode_step). */
+/* Quantize fp32 states S [n, H, dk, dv] into the slots slot_ids[n] of a pool (impact,
+ * row_bits: as for oracle_decode_step). */
 long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_slots, uint8_t *pool,
-                      const int32_t *slot_ids, int n, const float *S, int nthreads, const float *impact)
+                      const int32_t *slot_ids, int n, const float *S, int nthreads, const float *impact,
+                      const int32_t *row_bits)
 {
     long *offsets = (long *)malloc((size_t)H * sizeof(long));
-    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets, row_bits);
     long clipped = 0;
     int bad = 0;
     long items = (long)n * H;
@@ -489,11 +657,14 @@ long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_s
         }
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
-        if (impact)
+        const int32_t *rb = head_bits[h] ? NULL : row_bits + (long)h * dk;
+        if (rb)
+            clipped += oracle_rows_quantize(dk, dv, rb, S + it * ne, Q, r, c);
+        else if (impact)
             (void)oracle_quantize_impact(head_bits[h], dk, dv, S + it * ne, impact + (long)h * dk, Q, r, c);
         else
             clipped += oracle_quantize(head_bits[h], dk, dv, S + it * ne, Q, r, c);
-        write_block(pool + (long)slot * stride + offsets[h], head_bits[h], dk, dv, Q, r, c);
+        write_block(pool + (long)slot * stride + offsets[h], head_bits[h], rb, dk, dv, Q, r, c);
         free(Q); free(r); free(c);
     }
     free(offsets);
@@ -502,10 +673,10 @@ long oracle_pool_load(int H, int dk, int dv, const int32_t *head_bits, int num_s
 
 /* Dequantize the slots slot_ids[n] of a pool into S [n, H, dk, dv] (fp32). */
 int oracle_pool_dump(int H, int dk, int dv, const int32_t *head_bits, int num_slots, const uint8_t *pool,
-                     const int32_t *slot_ids, int n, float *S, int nthreads)
+                     const int32_t *slot_ids, int n, float *S, int nthreads, const int32_t *row_bits)
 {
     long *offsets = (long *)malloc((size_t)H * sizeof(long));
-    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets);
+    long stride = oracle_head_offsets(H, head_bits, dk, dv, offsets, row_bits);
     int bad = 0;
     long items = (long)n * H;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads) reduction(| : bad)
@@ -524,7 +695,8 @@ int oracle_pool_dump(int H, int dk, int dv, const int32_t *head_bits, int num_sl
         int32_t *Q = (int32_t *)malloc((size_t)ne * sizeof(int32_t));
         float *r = (float *)malloc(4L * dk), *c = (float *)malloc(4L * dv);
         double *Sd = (double *)malloc((size_t)ne * sizeof(double));
-        read_block(pool + (long)slot * stride + offsets[h], head_bits[h], dk, dv, Q, r, c);
+        read_block(pool + (long)slot * stride + offsets[h], head_bits[h],
+                   head_bits[h] ? NULL : row_bits + (long)h * dk, dk, dv, Q, r, c);
         oracle_dequantize(dk, dv, Q, r, c, Sd);
         for (long e = 0; e < ne; e++) S[it * ne + e] = (float)Sd[e];
         free(Q); free(r); free(c); free(Sd);

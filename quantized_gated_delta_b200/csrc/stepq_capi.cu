@@ -49,6 +49,11 @@ void free_pool(stepq_pool *p)
     cudaFree(p->d_order);
     cudaFree(p->d_flag);
     cudaFree(p->d_impact);
+    cudaFree(p->d_blk);
+    cudaFree(p->d_rn8);
+    cudaFree(p->d_rn4);
+    cudaFree(p->d_rpb);
+    cudaFree(p->d_perm);
     delete p;
 }
 
@@ -63,13 +68,19 @@ const char *stepq_status_string(int status)
     case STEPQ_INVALID_ARG: return "invalid argument";
     case STEPQ_OUT_OF_MEMORY: return "out of memory";
     case STEPQ_CUDA_ERROR: return "CUDA error";
-    case STEPQ_UNSUPPORTED: return "unsupported configuration (d_k = d_v = 128, bits in {4, 6, 8, 16})";
+    case STEPQ_UNSUPPORTED: return "unsupported configuration (d_k = d_v = 128, bits in {4, 6, 8, 16}, row bits in {4, 6, 8})";
     case STEPQ_DEVICE_FLAG: return "device flag set (bad slot id or kernel wait timeout)";
     default: return "unknown status";
     }
 }
 
-int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
+}  // extern "C"
+
+namespace {
+
+// Pool creation; row_bits (host [H, d_k] or null) gives the per-key-row widths of the heads of
+// width 0.
+int create_pool(const stepq_pool_desc *desc, const uint8_t *row_bits, stepq_pool **out)
 {
     if (!desc || !out || !desc->head_bits) return STEPQ_INVALID_ARG;
     *out = nullptr;
@@ -79,9 +90,18 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     if (desc->gate_mode != STEPQ_GATE_GDN && desc->gate_mode != STEPQ_GATE_KDA) return STEPQ_INVALID_ARG;
     if (desc->in_dtype != STEPQ_DTYPE_F32 && desc->in_dtype != STEPQ_DTYPE_BF16) return STEPQ_INVALID_ARG;
     if (desc->d_k != stepq::DK || desc->d_v != stepq::DV) return STEPQ_UNSUPPORTED;
+    bool any_rows = false;
     for (int h = 0; h < desc->num_heads; ++h) {
         const int b = desc->head_bits[h];
-        if (b != 4 && b != 6 && b != 8 && b != 16) return STEPQ_UNSUPPORTED;
+        if (b == 0 && row_bits) {
+            any_rows = true;
+            for (int i = 0; i < stepq::DK; ++i) {
+                const int rb = row_bits[h * stepq::DK + i];
+                if (rb != 4 && rb != 6 && rb != 8) return STEPQ_UNSUPPORTED;
+            }
+        } else if (b != 4 && b != 6 && b != 8 && b != 16) {
+            return STEPQ_UNSUPPORTED;
+        }
     }
     stepq_pool *p = new (std::nothrow) stepq_pool();
     if (!p) return STEPQ_OUT_OF_MEMORY;
@@ -92,14 +112,40 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     p->in_dtype = desc->in_dtype;
     p->bits.assign(desc->head_bits, desc->head_bits + p->H);
     p->offs.resize(p->H);
+    std::vector<int32_t> blk(p->H);
+    if (any_rows) {
+        p->rn8.assign(p->H, 0);
+        p->rn4.assign(p->H, 0);
+        p->rpb.assign(p->H, 0);
+        p->perm.assign(size_t(p->H) * stepq::DK, 0);
+    }
     long long off = 0;
     for (int h = 0; h < p->H; ++h) {
         p->offs[h] = off;
-        off += block_bytes(p->bits[h]);
+        if (p->bits[h] == 0) {
+            // rows stored 8-bit, then 4-bit, then 6-bit (ascending key row in each group);
+            // panels padded to 16 bytes
+            const uint8_t *rb = row_bits + h * stepq::DK;
+            int n[3] = {0, 0, 0}, pos = 0;
+            const int widths[3] = {8, 4, 6};
+            for (int wdt = 0; wdt < 3; ++wdt)
+                for (int i = 0; i < stepq::DK; ++i)
+                    if (rb[i] == widths[wdt]) {
+                        p->perm[size_t(h) * stepq::DK + pos++] = uint8_t(i);
+                        ++n[wdt];
+                    }
+            p->rn8[h] = uint8_t(n[0]);
+            p->rn4[h] = uint8_t(n[1]);
+            p->rpb[h] = (16 * n[0] + 8 * n[1] + 12 * n[2] + 15) / 16 * 16;
+            blk[h] = stepq::NPANEL * p->rpb[h] + 4 * stepq::DK + 4 * stepq::DV;
+        } else {
+            blk[h] = block_bytes(p->bits[h]);
+        }
+        off += blk[h];
         if (p->bits[h] == 16)
             ++p->npiv;
-        else if (block_bytes(p->bits[h]) > p->max_block)
-            p->max_block = block_bytes(p->bits[h]);
+        else if (blk[h] > p->max_block)
+            p->max_block = blk[h];
     }
     p->slot_stride = off;
     p->total = off * (long long)p->num_slots;
@@ -114,11 +160,23 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     if (e == cudaSuccess) e = cudaMemset(p->d_flag, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemcpy(p->d_offs, p->offs.data(), sizeof(long long) * p->H, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_bits, p->bits.data(), size_t(p->H), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && any_rows) {
+        e = cudaMalloc(&p->d_blk, sizeof(int32_t) * p->H);
+        if (e == cudaSuccess) e = cudaMalloc(&p->d_rn8, size_t(p->H));
+        if (e == cudaSuccess) e = cudaMalloc(&p->d_rn4, size_t(p->H));
+        if (e == cudaSuccess) e = cudaMalloc(&p->d_rpb, sizeof(int32_t) * p->H);
+        if (e == cudaSuccess) e = cudaMalloc(&p->d_perm, p->perm.size());
+        if (e == cudaSuccess) e = cudaMemcpy(p->d_blk, blk.data(), sizeof(int32_t) * p->H, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = cudaMemcpy(p->d_rn8, p->rn8.data(), size_t(p->H), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = cudaMemcpy(p->d_rn4, p->rn4.data(), size_t(p->H), cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = cudaMemcpy(p->d_rpb, p->rpb.data(), sizeof(int32_t) * p->H, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) e = cudaMemcpy(p->d_perm, p->perm.data(), p->perm.size(), cudaMemcpyHostToDevice);
+    }
     if (e == cudaSuccess) {
-        // the decode kernel visits heads grouped by bit width (stable within a width); the
-        // FP16 pivot heads come last and go to their own kernel
+        // the decode kernel visits heads grouped by bit width (stable within a width): 4, 6,
+        // 8, per-key-row widths; the FP16 pivot heads come last and go to their own kernel
         std::vector<int32_t> order;
-        for (int w : {4, 6, 8, 16})
+        for (int w : {4, 6, 8, 0, 16})
             for (int h = 0; h < p->H; ++h)
                 if (p->bits[h] == w) order.push_back(h);
         e = cudaMemcpy(p->d_order, order.data(), sizeof(int32_t) * p->H, cudaMemcpyHostToDevice);
@@ -131,6 +189,18 @@ int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out)
     }
     *out = p;
     return STEPQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int stepq_pool_create(const stepq_pool_desc *desc, stepq_pool **out) { return create_pool(desc, nullptr, out); }
+
+int stepq_pool_create_rows(const stepq_pool_desc *desc, const uint8_t *row_bits, stepq_pool **out)
+{
+    if (!row_bits) return STEPQ_INVALID_ARG;
+    return create_pool(desc, row_bits, out);
 }
 
 int stepq_pool_destroy(stepq_pool *pool)

@@ -53,7 +53,8 @@ constexpr unsigned kFull = 0xffffffffu;
 struct StageMeta {
     long long dst;                  // byte offset of the head block in the pool
     int valid;
-    int bits;
+    int bits;                       // 4, 6, 8, or 0: per-key-row widths
+    int head;
 };
 
 struct DecodeArgs {
@@ -63,7 +64,14 @@ struct DecodeArgs {
     const uint8_t *head_bits;
     const int32_t *head_order;      // processing order of the heads (grouped by bit width)
     int num_slots, H, Hk, group;
-    int nh4, nh6;                   // heads of width 4 and 6 (visited first, in that order)
+    int nh4, nh6, nh8;              // heads of width 4, 6 and 8 (visited in that order, then the
+                                    // heads with per-key-row widths)
+    // heads with per-key-row widths (width 0): block bytes, rows of width 8 and 4 (stored
+    // first, in that order; the rest are 6-bit), padded panel bytes, stored row -> key row
+    const int32_t *head_blk;
+    const uint8_t *row_n8, *row_n4;
+    const int32_t *row_pb;
+    const uint8_t *row_perm;
     int Hq;                         // quantized heads: the first Hq entries of head_order
     const float *impact;            // [H, d_k] normalized row-impact weights (impact fit), or null
     const int32_t *slot_ids;
@@ -113,18 +121,19 @@ struct Cursor {
 // Per-row weights of a state held in a stage, built by thread t (128 <= t < 256) for row
 // t - 128, and the share of k.q of warps 4..7.
 template <int GATE, typename TIn>
-__device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs &a, int bits, float alpha_s,
-                                          Scratch &sc, int t)
+__device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs &a, int bits, int head,
+                                          float alpha_s, Scratch &sc, int t)
 {
-    const int i = t - 128;
-    const float *r = reinterpret_cast<const float *>(stage + codes_bytes(bits));
+    const int i = t - 128;                          // stored row (the key row unless bits == 0)
+    const float *r = reinterpret_cast<const float *>(stage + (bits ? codes_bytes(bits) : 8 * a.row_pb[head]));
+    const int key = bits ? i : int(a.row_perm[head * DK + i]);
     const TIn *qs = reinterpret_cast<const TIn *>(stage + a.blk_cap);
     const TIn *ks = reinterpret_cast<const TIn *>(stage + a.blk_cap + kIoBytes);
     const TIn *as = reinterpret_cast<const TIn *>(stage + a.blk_cap + 3 * kIoBytes);
-    const float al = (GATE == STEPQ_GATE_KDA) ? to_f32(as[i]) : alpha_s;
+    const float al = (GATE == STEPQ_GATE_KDA) ? to_f32(as[key]) : alpha_s;
     const float rho = al * r[i];
-    const float k = to_f32(ks[i]);
-    const float q = to_f32(qs[i]);
+    const float k = to_f32(ks[key]);
+    const float q = to_f32(qs[key]);
     const float rk = rho * k, rq = rho * q;
     sc.wlo[i] = make_float4(rk, rk, rq, rq);
     sc.whi[i] = make_float4(rq, rq, rk, rk);
@@ -150,24 +159,46 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
                                             TIn alpha_next_raw, bool ok)
 {
     uint8_t *stage = stages + (i % kStages) * a.stage_bytes;
-    constexpr int QM = qmax_of(BITS);
-    constexpr float MAG = kTwo23 + float(1 << (BITS - 1));
+    // BITS == 0: per-key-row widths (rows stored 8-bit, 4-bit, 6-bit; codes unscaled)
+    constexpr int QM = BITS ? qmax_of(BITS) : 1;
+    constexpr float MAG = kTwo23 + float(1 << ((BITS ? BITS : 1) - 1));
     constexpr int BI = BITS == 4 ? 0 : BITS == 6 ? 1 : 2;
     const int lane = ix.lane;
     const int panel = ix.panel;
     const bool upper = (lane & 16) != 0;            // lanes holding the q-weighted sums first
     const int col = lane & 15;                      // the column this lane finalizes
+    const int head = int(bh % a.H);
+    int n8 = 0, n4 = 0, pb = panel_bytes(BITS ? BITS : 4);
+    if constexpr (BITS == 0) {
+        n8 = a.row_n8[head];
+        n4 = a.row_n4[head];
+        pb = a.row_pb[head];
+    }
+    const int cbytes = BITS ? codes_bytes(BITS) : 8 * pb;
 
     uint8_t *codes = stage;
-    float *r_io = reinterpret_cast<float *>(stage + codes_bytes(BITS));
+    float *r_io = reinterpret_cast<float *>(stage + cbytes);
     float *c_io = r_io + DK;
     const TIn *vs = reinterpret_cast<const TIn *>(stage + a.blk_cap + 2 * kIoBytes);
 
     // ---- codes of the thread's 4 rows x 16 columns (times their position scale), exact floats
     float T[kRows][PANEL];
 #pragma unroll
-    for (int m = 0; m < kRows; ++m)
-        load_codes<BITS>(codes + panel * panel_bytes(BITS) + ix.row(m) * seg_bytes(BITS), T[m]);
+    for (int m = 0; m < kRows; ++m) {
+        if constexpr (BITS == 0) {
+            const int p = ix.row(m);
+            const uint8_t *seg = codes + panel * pb + row_seg_off(p, n8, n4);
+            const int wdt = row_width(p, n8, n4);
+            if (wdt == 8)
+                load_codes_unscaled<8>(seg, T[m]);
+            else if (wdt == 4)
+                load_codes_unscaled<4>(seg, T[m]);
+            else
+                load_codes_unscaled<6>(seg, T[m]);
+        } else {
+            load_codes<BITS>(codes + panel * panel_bytes(BITS) + ix.row(m) * seg_bytes(BITS), T[m]);
+        }
+    }
 
     // A zero column factor means a zero column whatever its codes (a fresh pool holds
     // nonzero codes under zero scales): clear those codes.  Warp-uniform and rare.
@@ -181,7 +212,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         }
     }
     // column factor of the scaled codes (a zero column behaves as c = 1: S = T = k d)
-    const float cprime = (cj == 0.0f ? 1.0f : cj) * sc.invpos[BI][col];
+    const float cprime = (cj == 0.0f ? 1.0f : cj) * (BITS ? sc.invpos[BI][col] : 1.0f);
 
     // ---- column dot products over the thread's rows (column pairs, f32x2), then over the
     // warp: lane bit 4 first (select-free: the partner's second sum is this lane's first
@@ -231,7 +262,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
             T[m][j + 1] = t.y;
         }
     }
-    if constexpr (IMPACT)
+    if constexpr (IMPACT && BITS != 0)          // heads with per-row widths keep the clip-free fit
         return refit_impact<GATE, TIn, BITS>(T, stages, i, has_next, a, sc, ix, tid, int(bh % a.H), cprime,
                                              alpha_next_raw, ok, r_io, c_io, codes);
     // column maxima: over the thread's rows, then a warp-wide max per column; the 16
@@ -283,14 +314,23 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         const float4 u = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride);
         const float4 v = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride + 4);
         const float mr = fmaxf(max3(u.x, u.y, u.z), max3(max3(u.w, v.x, v.y), v.z, v.w));
-        const float r = div_const<QM>(mr);
+        float r;
+        if constexpr (BITS == 0) {
+            const int wdt = row_width(tid, n8, n4);
+            r = div_refined(mr, float(qmax_of(wdt)));
+            const float ir = r >= FLT_MIN ? rcp_refined(r) : 0.0f;
+            const float mag = kTwo23 + float(1 << (wdt - 1));
+            sc.fit[tid] = make_float4(ir, ir, mag, mag);
+        } else {
+            r = div_const<QM>(mr);
+            const float ir = r >= FLT_MIN ? rcp_refined(r) : 0.0f;
+            sc.ir[tid] = make_float2(ir, ir);
+        }
         r_io[tid] = r;
         tiny = r > 0.0f && r < FLT_MIN;
-        const float ir = r >= FLT_MIN ? rcp_refined(r) : 0.0f;
-        sc.ir[tid] = make_float2(ir, ir);
     } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
         row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
-                             to_f32(alpha_next_raw), sc, tid);
+                             sc.meta[(i + 1) % kStages].head, to_f32(alpha_next_raw), sc, tid);
     }
     const bool any_tiny = __syncthreads_or(tiny);
 
@@ -299,11 +339,18 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
 #pragma unroll
     for (int m = 0; m < kRows; ++m) {
         const int row = ix.row(m);
-        const float2 ir = sc.ir[row];
+        float2 ir, mag2 = make_float2(MAG, MAG);
+        if constexpr (BITS == 0) {
+            const float4 f = sc.fit[row];
+            ir = make_float2(f.x, f.y);
+            mag2 = make_float2(f.z, f.w);
+        } else {
+            ir = sc.ir[row];
+        }
         uint32_t u[PANEL];
 #pragma unroll
         for (int j = 0; j < PANEL; j += 2) {
-            const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), ir, make_float2(MAG, MAG));
+            const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), ir, mag2);
             u[j] = __float_as_uint(f.x);
             u[j + 1] = __float_as_uint(f.y);
         }
@@ -313,19 +360,30 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
             if (r > 0.0f && r < FLT_MIN) {
                 const float irs = rcp_refined(r * 0x1p64f);
 #pragma unroll
-                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(fmaf(T[m][j] * 0x1p64f, irs, MAG));
+                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(fmaf(T[m][j] * 0x1p64f, irs, mag2.x));
             }
         }
-        pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
+        if constexpr (BITS == 0) {
+            uint8_t *seg = codes + panel * pb + row_seg_off(row, n8, n4);
+            const int wdt = row_width(row, n8, n4);
+            if (wdt == 8)
+                pack_seg<8>(u, seg);
+            else if (wdt == 4)
+                pack_seg<4>(u, seg);
+            else
+                pack_seg<6>(u, seg);
+        } else {
+            pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
+        }
     }
     // each warp stores its panel of codes and its slice of c (warp 0 also r)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
         uint8_t *dst = a.pool + sc.meta[i % kStages].dst;
-        bulk_s2g(dst + panel * panel_bytes(BITS), codes + panel * panel_bytes(BITS), panel_bytes(BITS));
-        bulk_s2g(dst + codes_bytes(BITS) + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
-        if (panel == 0) bulk_s2g(dst + codes_bytes(BITS), r_io, 4 * DK);
+        bulk_s2g(dst + panel * pb, codes + panel * pb, uint32_t(pb));
+        bulk_s2g(dst + cbytes + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
+        if (panel == 0) bulk_s2g(dst + cbytes, r_io, 4 * DK);
     }
     return true;
 }
@@ -388,7 +446,7 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
         fence_proxy_async_smem();                  // r is bulk-stored from the stage by warp 0
     } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
         row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
-                             to_f32(alpha_next_raw), sc, tid);
+                             sc.meta[(i + 1) % kStages].head, to_f32(alpha_next_raw), sc, tid);
     }
     __syncthreads();
 
@@ -514,11 +572,12 @@ struct ItemLoop {
             mbar_arrive(&sc.full[st]);
         } else {
             const int bits = sc.hbits[h];
-            const uint32_t bb = uint32_t(block_bytes(bits));
+            const uint32_t bb = bits ? uint32_t(block_bytes(bits)) : uint32_t(a.head_blk[h]);
             const long long bh = (long long)b * a.H + h;
             const long long kqrow = (long long)b * a.Hk + g;
             mt.valid = 1;
             mt.bits = bits;
+            mt.head = h;
             mt.dst = (long long)slot * a.slot_stride + sc.hoff[h];
             const uint32_t io = DK * esz;
             mbar_arrive_expect_tx(&sc.full[st], bb + 3 * io + (GATE == STEPQ_GATE_KDA ? io : 0u));
@@ -570,7 +629,7 @@ struct ItemLoop {
                 if (alive) {
                     const StageMeta mn = sc.meta[(i + 1) % kStages];
                     if (has_next && mn.valid && tid >= DK)
-                        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits,
+                        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits, mn.head,
                                              to_f32(alpha_raw), sc, tid);
                     __syncthreads();
                 }
@@ -607,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     };
     const int end4 = class_end((long long)a.nh4 * a.n);
     const int end6 = class_end((long long)(a.nh4 + a.nh6) * a.n);
+    const int end8 = class_end((long long)(a.nh4 + a.nh6 + a.nh8) * a.n);
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -642,12 +702,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     {
         const StageMeta m0 = sc.meta[0];
         const float al0 = (GATE == STEPQ_GATE_GDN) ? to_f32(alpha_g[L.bh_cur]) : 1.0f;
-        if (m0.valid && tid >= DK) row_table<GATE, TIn>(stages, a, m0.bits, al0, sc, tid);
+        if (m0.valid && tid >= DK) row_table<GATE, TIn>(stages, a, m0.bits, m0.head, al0, sc, tid);
     }
     __syncthreads();
 
     int i = 0;
-    const bool done = L.template run<4>(i, end4) && L.template run<6>(i, end6) && L.template run<8>(i, count);
+    const bool done = L.template run<4>(i, end4) && L.template run<6>(i, end6) && L.template run<8>(i, end8) &&
+                      L.template run<0>(i, count);
     const int lane = tid & 31;
     if (lane == 0) bulk_wait_all();
     if (tid == 0 && !done) {
@@ -815,10 +876,11 @@ cudaError_t upload_tables()
 
 void count_widths(const uint8_t *bits, int H, DecodeArgs &a)
 {
-    a.nh4 = a.nh6 = 0;
+    a.nh4 = a.nh6 = a.nh8 = 0;
     for (int h = 0; h < H; ++h) {
         a.nh4 += bits[h] == 4;
         a.nh6 += bits[h] == 6;
+        a.nh8 += bits[h] == 8;
     }
 }
 
@@ -862,6 +924,11 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.stage_bytes = p->stage_bytes;
     a.Hq = p->H - p->npiv;
     a.impact = p->d_impact;
+    a.head_blk = p->d_blk;
+    a.row_n8 = p->d_rn8;
+    a.row_n4 = p->d_rn4;
+    a.row_pb = p->d_rpb;
+    a.row_perm = p->d_perm;
     // items are dealt round-robin in head-major order, so the CTAs resident at any moment
     // work on one or two heads (one bit width: one code path in the instruction caches)
     const long long total = (long long)n * a.Hq;
@@ -1059,6 +1126,9 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     a.group = H / desc->num_key_heads;
     a.Hq = H;
     a.impact = nullptr;
+    a.head_blk = nullptr;                   // every head here has a uniform width
+    a.row_n8 = a.row_n4 = a.row_perm = nullptr;
+    a.row_pb = nullptr;
     count_widths(bits, H, a);
     a.slot_ids = slot_ids;
     a.n = n;

@@ -23,6 +23,14 @@ struct stepq_pool {
     int32_t *d_order = nullptr;         // [H] head processing order (widths 4, 6, 8, then pivots)
     int *d_flag = nullptr;              // sticky device flag (STEPQ_FLAG_* bits)
     float *d_impact = nullptr;          // [H, d_k] normalized row-impact weights (impact fit), or null
+    // heads with per-key-row widths (width 0 in bits): rows of width 8 and 4, padded panel
+    // bytes, block bytes, stored row -> key row; null when the pool has none
+    std::vector<uint8_t> rn8, rn4;      // [H]
+    std::vector<int32_t> rpb;           // [H]
+    std::vector<uint8_t> perm;          // [H * d_k]
+    int32_t *d_blk = nullptr;           // [H] block bytes of every head
+    uint8_t *d_rn8 = nullptr, *d_rn4 = nullptr, *d_perm = nullptr;
+    int32_t *d_rpb = nullptr;
     int decode_grid = 0;                // persistent CTAs for the decode kernel
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel
     int stage_bytes = 0;

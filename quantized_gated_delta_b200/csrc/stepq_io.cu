@@ -22,11 +22,11 @@ constexpr int kIoRpStride = 12;     // padded row stride of the row-maxima excha
 template <int ROWS, int BITS>
 __device__ __forceinline__ bool fit_quantize_pack(float (&S)[ROWS][PANEL], const TileIdx<ROWS> &ix,
                                                   float *rp, float *xc, uint8_t *codes_out,
-                                                  float *r_out, float *c_out, bool ok)
+                                                  float *r_out, float *c_out, bool ok,
+                                                  int n8 = 0, int n4 = 0, int pb = 0)
 {
+    // BITS == 0: per-key-row widths (stored rows 8-bit, 4-bit, 6-bit; panels of pb bytes)
     using L = Layout<ROWS>;
-    constexpr int QM = qmax_of(BITS);
-    constexpr float MAG = kTwo23 + float(1 << (BITS - 1));
 
     // column maxima: max_i |S_ij| over the thread's rows, then over the LP lanes of the panel
     float cm[PANEL];
@@ -88,7 +88,9 @@ __device__ __forceinline__ bool fit_quantize_pack(float (&S)[ROWS][PANEL], const
         const float4 a = *reinterpret_cast<const float4 *>(rp + row * kIoRpStride);
         const float4 b = *reinterpret_cast<const float4 *>(rp + row * kIoRpStride + 4);
         const float mr = max3(max3(a.x, a.y, a.z), max3(a.w, b.x, b.y), fmaxf(b.z, b.w));
-        const float r = mr / float(QM);
+        const int wdt = BITS ? BITS : row_width(row, n8, n4);
+        const float MAG = kTwo23 + float(1 << (wdt - 1));
+        const float r = mr / float(qmax_of(wdt));
         if (ix.panel == 0) r_out[row] = r;
         uint32_t u[PANEL];
         if (r >= FLT_MIN || r == 0.0f) {
@@ -107,7 +109,17 @@ __device__ __forceinline__ bool fit_quantize_pack(float (&S)[ROWS][PANEL], const
 #pragma unroll
             for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(S[m][j] / r + MAG);
         }
-        pack_seg<BITS>(u, codes_out + ix.panel * panel_bytes(BITS) + row * seg_bytes(BITS));
+        if constexpr (BITS == 0) {
+            uint8_t *seg = codes_out + ix.panel * pb + row_seg_off(row, n8, n4);
+            if (wdt == 8)
+                pack_seg<8>(u, seg);
+            else if (wdt == 4)
+                pack_seg<4>(u, seg);
+            else
+                pack_seg<6>(u, seg);
+        } else {
+            pack_seg<BITS>(u, codes_out + ix.panel * panel_bytes(BITS) + row * seg_bytes(BITS));
+        }
     }
     return true;
 }
@@ -191,6 +203,8 @@ struct IoArgs {
     const int32_t *slot_ids;
     int *flag;
     const float *impact;            // [H, d_k] normalized row-impact weights, or null (clip-free fit)
+    const uint8_t *row_n8, *row_n4, *row_perm;  // heads with per-key-row widths (see the pool)
+    const int32_t *row_pb;
 };
 
 template <int BITS>
@@ -227,6 +241,23 @@ __global__ void __launch_bounds__(256) load_fp32_kernel(const IoArgs a, const fl
     const float *Si = S + it * DK * DV;
     const TileIdx<4> ix(threadIdx.x);
     switch (a.head_bits[h]) {
+    case 0: {
+        // per-key-row widths: stored row p holds key row perm[p]
+        const int n8 = a.row_n8[h], n4 = a.row_n4[h], pb = a.row_pb[h];
+        float T[4][PANEL];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int key = a.row_perm[h * DK + ix.row(m)];
+#pragma unroll
+            for (int j = 0; j < PANEL; j += 4) {
+                const float4 t = *reinterpret_cast<const float4 *>(Si + key * DV + ix.panel * PANEL + j);
+                T[m][j] = t.x; T[m][j + 1] = t.y; T[m][j + 2] = t.z; T[m][j + 3] = t.w;
+            }
+        }
+        float *r_out = reinterpret_cast<float *>(blk + NPANEL * pb);
+        fit_quantize_pack<4, 0>(T, ix, rp, xc, blk, r_out, r_out + DK, true, n8, n4, pb);
+        break;
+    }
     case 4: load_fp32_item<4>(a, blk, Si, ix, rp, xc, h); break;
     case 6: load_fp32_item<6>(a, blk, Si, ix, rp, xc, h); break;
     case 8: load_fp32_item<8>(a, blk, Si, ix, rp, xc, h); break;
@@ -277,6 +308,30 @@ __global__ void __launch_bounds__(256) dump_fp32_kernel(const IoArgs a, float *S
     float *Si = S + it * DK * DV;
     const TileIdx<4> ix(threadIdx.x);
     switch (a.head_bits[h]) {
+    case 0: {
+        const int n8 = a.row_n8[h], n4 = a.row_n4[h], pb = a.row_pb[h];
+        const float *r = reinterpret_cast<const float *>(blk + NPANEL * pb);
+        const float *c = r + DK;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int p = ix.row(m);
+            const int key = a.row_perm[h * DK + p];
+            const int wdt = row_width(p, n8, n4);
+            const uint8_t *seg = blk + ix.panel * pb + row_seg_off(p, n8, n4);
+            float f[PANEL];
+            if (wdt == 8)
+                load_codes_unscaled<8>(seg, f);
+            else if (wdt == 4)
+                load_codes_unscaled<4>(seg, f);
+            else
+                load_codes_unscaled<6>(seg, f);
+            const double rr = r[p];
+#pragma unroll
+            for (int j = 0; j < PANEL; ++j)       // (Q r) c in double, Q r exact
+                Si[key * DV + ix.panel * PANEL + j] = float(double(f[j]) * rr * double(c[ix.panel * PANEL + j]));
+        }
+        break;
+    }
     case 4: dump_fp32_item<4>(blk, Si, ix); break;
     case 6: dump_fp32_item<6>(blk, Si, ix); break;
     case 8: dump_fp32_item<8>(blk, Si, ix); break;
@@ -323,6 +378,10 @@ IoArgs io_args(const stepq_pool *p, const int32_t *slot_ids)
     a.slot_ids = slot_ids;
     a.flag = p->d_flag;
     a.impact = p->d_impact;
+    a.row_n8 = p->d_rn8;
+    a.row_n4 = p->d_rn4;
+    a.row_perm = p->d_perm;
+    a.row_pb = p->d_rpb;
     return a;
 }
 

@@ -124,6 +124,31 @@ __device__ __forceinline__ void load_codes(const uint8_t *seg, float (&f)[PANEL]
     }
 }
 
+// codes of one row segment with the position scale removed (exact code values), for rows
+// whose widths differ inside one head: fma(f, 1/s, -(2^23 / s + 2^(b-1))) is exact
+template <int BITS>
+__device__ __forceinline__ void load_codes_unscaled(const uint8_t *seg, float (&f)[PANEL])
+{
+    unpack_seg<BITS>(seg, f);
+#pragma unroll
+    for (int p = 0; p < PANEL; p += 2) {
+        const float2 r = ffma2(make_float2(f[p], f[p + 1]),
+                               make_float2(1.0f / pos_scale(BITS, p), 1.0f / pos_scale(BITS, p + 1)),
+                               make_float2(-pos_bias(BITS, p) / pos_scale(BITS, p),
+                                           -pos_bias(BITS, p + 1) / pos_scale(BITS, p + 1)));
+        f[p] = r.x;
+        f[p + 1] = r.y;
+    }
+}
+
+// Per-key-row widths: a head's rows are stored 8-bit first, then 4-bit, then 6-bit; stored
+// row p has this width and starts this many bytes into its panel.
+__device__ __forceinline__ int row_width(int p, int n8, int n4) { return p < n8 ? 8 : p < n8 + n4 ? 4 : 6; }
+__device__ __forceinline__ int row_seg_off(int p, int n8, int n4)
+{
+    return p < n8 ? 16 * p : p < n8 + n4 ? 16 * n8 + 8 * (p - n8) : 16 * n8 + 8 * n4 + 12 * (p - n8 - n4);
+}
+
 // ---------------------------------------------------------------- pack one row segment
 // Input: raw bits of fma(x, 1, 2^23 + 2^(b-1)) results, i.e. 0x4B000000 + u.
 

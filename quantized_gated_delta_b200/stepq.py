@@ -28,7 +28,7 @@ EXPORTED = [
     "stepq_pool_load_fp32", "stepq_pool_load_packed", "stepq_pool_dump_fp32",
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
-    "stepq_allocate_bits_pivots", "stepq_pool_set_impact",
+    "stepq_allocate_bits_pivots", "stepq_pool_set_impact", "stepq_pool_create_rows",
 ]
 
 
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_allocate_bits": [P, P, I, P, I, ctypes.c_double, P],
         "stepq_allocate_bits_pivots": [P, P, I, P, I, ctypes.c_double, I, P],
         "stepq_pool_set_impact": [P, P],
+        "stepq_pool_create_rows": [ctypes.POINTER(stepq_pool_desc), P, ctypes.POINTER(P)],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
@@ -117,6 +118,21 @@ def stepq_pool_create(num_slots: int, head_bits, num_key_heads: int, gate_mode: 
                            hb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
     handle = ctypes.c_void_p()
     _check(load_library().stepq_pool_create(ctypes.byref(desc), ctypes.byref(handle)), "stepq_pool_create")
+    return handle.value
+
+
+def stepq_pool_create_rows(num_slots: int, head_bits, num_key_heads: int, row_bits, gate_mode: int = STEPQ_GATE_KDA,
+                           in_dtype: int = STEPQ_DTYPE_BF16, d_k: int = 128, d_v: int = 128) -> int:
+    """Pool whose heads of width 0 take per-key-row widths from row_bits [H, d_k]."""
+    hb = np.ascontiguousarray(head_bits, dtype=np.uint8)
+    rb = np.ascontiguousarray(row_bits, dtype=np.uint8)
+    if rb.shape != (len(hb), d_k):
+        raise ValueError("row_bits must be [H, d_k]")
+    desc = stepq_pool_desc(int(num_slots), len(hb), int(num_key_heads), d_k, d_v, gate_mode, in_dtype,
+                           hb.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    handle = ctypes.c_void_p()
+    _check(load_library().stepq_pool_create_rows(ctypes.byref(desc), rb.ctypes.data, ctypes.byref(handle)),
+           "stepq_pool_create_rows")
     return handle.value
 
 
@@ -226,11 +242,16 @@ class Pool:
     """Owning wrapper around a stepq_pool handle (device memory freed on close)."""
 
     def __init__(self, num_slots: int, head_bits, num_key_heads: int, gate_mode: int = STEPQ_GATE_GDN,
-                 in_dtype: int = STEPQ_DTYPE_BF16):
+                 in_dtype: int = STEPQ_DTYPE_BF16, row_bits=None):
         self.head_bits = np.ascontiguousarray(head_bits, dtype=np.uint8)
         self.num_slots, self.H, self.Hk = int(num_slots), len(self.head_bits), int(num_key_heads)
         self.gate_mode, self.in_dtype = gate_mode, in_dtype
-        self.handle = stepq_pool_create(num_slots, self.head_bits, num_key_heads, gate_mode, in_dtype)
+        self.handle = None
+        if row_bits is None:
+            self.handle = stepq_pool_create(num_slots, self.head_bits, num_key_heads, gate_mode, in_dtype)
+        else:
+            self.handle = stepq_pool_create_rows(num_slots, self.head_bits, num_key_heads, row_bits, gate_mode,
+                                                 in_dtype)
         self.slot_stride, self.total_bytes = stepq_pool_bytes(self.handle)
 
     def close(self):

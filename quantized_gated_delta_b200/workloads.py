@@ -73,7 +73,8 @@ class Workload:
     n_pivots: int = 0         # FP16 pivot heads per layer chosen by the allocator
     layers: int = 1
     warmup_steps: int = 32
-    kda_mu: np.ndarray | None = None      # [layers, H]
+    kda_mu: np.ndarray | None = None      # [layers, H], or [layers, H, dk] (per-channel gates)
+    row_half_life: np.ndarray | None = None   # [layers, H, dk]: per-key-row widths (KDA, unit = key row)
     dk: int = 128
     dv: int = 128
 
@@ -88,6 +89,22 @@ def _rng(seed: int, *key: int) -> np.random.Generator:
 
 def _softplus(x):
     return np.logaddexp(0.0, x)
+
+
+def kda_mu_for_half_lives(h: np.ndarray) -> np.ndarray:
+    """kda_mu_for_half_life over an array (vectorised bisection on the same quadrature)."""
+    nodes, weights = np.polynomial.hermite_e.hermegauss(64)
+    weights = weights / weights.sum()
+    target = math.log(2.0) / np.asarray(h, dtype=np.float64)
+    lo = np.full(target.shape, -40.0)
+    hi = np.full(target.shape, 10.0)
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        ms = (_softplus(mid[..., None] + nodes) * weights).sum(-1)
+        big = ms > target
+        hi = np.where(big, mid, hi)
+        lo = np.where(big, lo, mid)
+    return 0.5 * (lo + hi)
 
 
 def kda_mu_for_half_life(h: float) -> float:
@@ -126,10 +143,17 @@ def make_workload(config: int, variant: str = "mixed6", batch: int | None = None
     smallest nonzero share at 32 heads (the pages keep 1.39% of the heads in FP16)
     5  36-layer GDN stack: H=32, Hk=16, T=32 per layer, B in {64, 256, 1024} (``batch``), bf16
     """
-    if variant not in ("mixed6", "mixed6p", "uniform4") or (variant == "uniform4" and config != 4) \
-            or (variant == "mixed6p" and config not in (2, 3, 4)):
+    if variant not in ("mixed6", "mixed6p", "uniform4", "rowbits") or (variant == "uniform4" and config != 4) \
+            or (variant == "mixed6p" and config not in (2, 3, 4)) or (variant == "rowbits" and config != 3):
         raise ValueError("variant %r of workload %r" % (variant, config))
     w = _make_workload(config, variant, batch)
+    if variant == "rowbits":
+        # every key channel its own mean gate: half-lives log-uniform over [2, 4096] per
+        # (head, channel); the allocation unit is the key row
+        rhl = np.exp(_rng(w.seed, 0, 6000).uniform(math.log(2.0), math.log(4096.0), (1, w.H, w.dk)))
+        w.row_half_life = rhl
+        w.kda_mu = kda_mu_for_half_lives(rhl)
+        w.name += "_rowbits"
     if variant == "mixed6p":
         w.n_pivots = 1
         w.name += "_p"
@@ -199,7 +223,8 @@ def step_inputs(w: Workload, t: int, phase: int = PHASE_RUN, layer: int = 0) -> 
     if w.gate_mode == GATE_GDN:
         alpha = np.broadcast_to((2.0 ** (-1.0 / w.half_life[layer])).astype(f32), (B, H))
     else:
-        x = r.standard_normal((B, H, dk)) + w.kda_mu[layer][None, :, None]
+        mu = np.asarray(w.kda_mu[layer])
+        x = r.standard_normal((B, H, dk)) + (mu[None, :, None] if mu.ndim == 1 else mu[None, :, :])
         alpha = np.exp(-_softplus(x))
     out = dict(q=q, k=k, v=v, beta=beta, alpha=alpha)
     for key in out:

@@ -31,11 +31,29 @@ def head_bits(w: W.Workload, layer: int = 0) -> np.ndarray:
     """Fixed widths of the workload, else the oracle's lifetime-aware allocation."""
     if w.head_bits is not None:
         return np.asarray(w.head_bits[layer], dtype=np.int32)
+    if w.row_half_life is not None:
+        return np.zeros(w.H, dtype=np.int32)          # every head: per-key-row widths
     if w.n_pivots:
         bits, _ = O.allocate_bits_pivots(list(w.half_life[layer]), None, [4, 6, 8], w.avg_bits, w.n_pivots)
         return np.asarray(bits, dtype=np.int32)
     bits, _ = O.allocate_bits_dp(list(w.half_life[layer]), None, [4, 6, 8], w.avg_bits)
     return np.asarray(bits, dtype=np.int32)
+
+
+_ROW_BITS_CACHE = {}
+
+
+def row_bits(w: W.Workload, layer: int = 0):
+    """Per-key-row widths [H, dk] of a workload whose allocation unit is the key row, from
+    the oracle's exact allocation over the layer's H * dk rows (None otherwise)."""
+    if w.row_half_life is None:
+        return None
+    key = (w.name, w.seed, layer)
+    if key not in _ROW_BITS_CACHE:
+        hl = list(np.asarray(w.row_half_life[layer], dtype=np.float64).ravel())
+        bits, _ = O.allocate_bits_dp_vec(hl, None, [4, 6, 8], w.avg_bits)
+        _ROW_BITS_CACHE[key] = np.asarray(bits, dtype=np.int32).reshape(w.H, w.dk)
+    return _ROW_BITS_CACHE[key]
 
 
 def sub_inputs(x: dict, idx) -> dict:
@@ -45,7 +63,7 @@ def sub_inputs(x: dict, idx) -> dict:
 def oracle_pool_with_warmup(w: W.Workload, bits, req_idx, layer: int = 0) -> O.OraclePool:
     """Oracle pool whose slots slot_ids[req_idx] hold the quantized state reached after the
     workload's FP32 warm-up steps (unquantized steps from zero, fp32-stored)."""
-    pool = O.OraclePool(w.num_slots, bits, w.Hk, w.gate_mode)
+    pool = O.OraclePool(w.num_slots, bits, w.Hk, w.gate_mode, row_bits=row_bits(w, layer))
     req_idx = np.asarray(req_idx)
     S = np.zeros((len(req_idx), w.H, w.dk, w.dv))
     for t in range(w.warmup_steps):
@@ -82,15 +100,16 @@ def fp16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(key(a) - key(b))
 
 
-def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv=128) -> dict:
-    """Compare slot images [n, slot_stride] head by head (FP16 pivot heads by binary16 ulps)."""
-    offs, stride = O.head_offsets(bits, dk, dv)
+def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv=128, row_bits=None) -> dict:
+    """Compare slot images [n, slot_stride] head by head (FP16 pivot heads by binary16 ulps;
+    heads of width 0 by their per-key-row widths row_bits [H, dk])."""
+    offs, stride = O.head_offsets(bits, dk, dv, row_bits)
     res = dict(max_code_diff=0, flips=0, elements=0, r_ulp=0, c_ulp=0, byte_equal=True,
                pivot_ulp=0, pivot_flips=0, pivot_elements=0)
     for s in range(gpu_bytes.shape[0]):
         for h, b in enumerate(bits):
             o = int(offs[h])
-            n = O.block_bytes(int(b), dk, dv)
+            n = O.block_bytes(int(b), dk, dv) if int(b) else O.rows_block_bytes(row_bits[h], dv)
             g, r = gpu_bytes[s, o:o + n], ora_bytes[s, o:o + n]
             if int(b) == 16:
                 d16 = fp16_ulp_diff(O.pivot_state(g, dk, dv), O.pivot_state(r, dk, dv))
@@ -103,8 +122,12 @@ def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv
                 res["elements"] += dk * dv
                 continue
             res["byte_equal"] = False
-            Qg, rg, cg = O.split_block(g, int(b), dk, dv)
-            Qo, ro, co = O.split_block(r, int(b), dk, dv)
+            if int(b):
+                Qg, rg, cg = O.split_block(g, int(b), dk, dv)
+                Qo, ro, co = O.split_block(r, int(b), dk, dv)
+            else:
+                Qg, rg, cg = O.rows_split_block(g, row_bits[h], dv)
+                Qo, ro, co = O.rows_split_block(r, row_bits[h], dv)
             d = np.abs(Qg - Qo)
             res["max_code_diff"] = max(res["max_code_diff"], int(d.max()))
             res["flips"] += int((d > 0).sum())

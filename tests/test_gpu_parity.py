@@ -341,6 +341,7 @@ CASES = [
     (4, "mixed6p", None, 0, 6, 32),
     (3, "mixed6p", None, 0, 4, 32),
     (2, "mixed6p", None, 0, 6, 32),
+    (3, "rowbits", None, 0, 4, 32),
     (5, "mixed6", 64, 17, 3, 32),
     (5, "mixed6", 256, 17, 3, 32),
     (5, "mixed6", 1024, 0, 3, 32),
@@ -362,7 +363,8 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
     sub = W.sample_requests(w, nsample)
     sub_slots = w.slot_ids[sub]
     op = PH.oracle_pool_with_warmup(w, bits, sub, layer)
-    gp = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    rb = PH.row_bits(w, layer)
+    gp = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype, row_bits=rb)
     load_bytes(gp, sub_slots, op.slot_bytes(sub_slots))
     all_slots = slots_t(w.slot_ids)
     num = den = 0.0
@@ -381,7 +383,7 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
         den += float(np.sum(yo.astype(np.float64) ** 2))
         worst["y"] = max(worst["y"], PH.y_max_rel(yg, yo))
         gb, ob = dump_bytes(gp, sub_slots), op.slot_bytes(sub_slots)
-        res = PH.compare_slots(gb, ob, bits)
+        res = PH.compare_slots(gb, ob, bits, row_bits=rb)
         flips += res["flips"]
         elements += res["elements"]
         pflips += res["pivot_flips"]
@@ -511,3 +513,44 @@ def test_impact_fit_trajectory_config4(S):
     op.decode_step(sub_slots, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"])
     res = PH.compare_slots(dump_bytes(gp, sub_slots), op.slot_bytes(sub_slots), bits)
     assert res["max_code_diff"] <= 1 and res["c_ulp"] <= PH.C_ULP
+
+
+# --------------------------------------------------------------------------- per-key-row widths
+
+def test_rowbits_heads_load_dump_and_step(S):
+    """Heads with per-key-row widths next to uniform heads: quantize-in, exact dump, and one
+    KDA bf16 step against the oracle (the usual single-step bars)."""
+    rng = np.random.default_rng(15)
+    H = 4
+    bits = [0, 8, 0, 4]
+    rb = np.stack([rng.choice([4, 6, 8], 128, p=[0.45, 0.35, 0.2]) for _ in range(H)]).astype(np.int32)
+    rb[2, :] = 4
+    rb[2, 3] = 6                                    # one 6-bit row among 4-bit rows
+    n = 3
+    st = random_states(rng, n, H)
+    ids = np.array([1, 3, 0], np.int32)
+    op = O.OraclePool(4, bits, 2, 1, row_bits=rb)
+    op.load_fp32(ids, st)
+    gp = S.Pool(4, bits, 2, S.STEPQ_GATE_KDA, S.STEPQ_DTYPE_BF16, row_bits=rb)
+    assert gp.slot_stride == op.slot_stride
+    gp.load_fp32(slots_t(ids), dev(st))
+    res = PH.compare_slots(dump_bytes(gp, ids), op.slot_bytes(ids), bits, row_bits=rb)
+    assert res["max_code_diff"] <= 1 and res["c_ulp"] == 0 and res["r_ulp"] <= PH.R_ULP, res
+    load_bytes(gp, ids, op.slot_bytes(ids))
+    out = torch.empty((n, H, 128, 128), dtype=torch.float32, device="cuda")
+    gp.dump_fp32(slots_t(ids), out)
+    assert np.array_equal(out.cpu().numpy(), op.dump_fp32(ids))
+    x = dict(q=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)])),
+             k=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)])),
+             v=W.round_bf16(rng.standard_normal((n, H, 128)).astype(f32)),
+             alpha=W.round_bf16(rng.uniform(0.6, 1, (n, H, 128)).astype(f32)),
+             beta=W.round_bf16(rng.uniform(0.1, 0.9, (n, H)).astype(f32)))
+    tx = {k_: dev(W.to_bf16_bits(v_).view(np.int16)) for k_, v_ in x.items()}
+    y = torch.empty((n, H, 128), device="cuda")
+    gp.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    assert gp.get_error() == 0
+    res = PH.compare_slots(dump_bytes(gp, ids), op.slot_bytes(ids), bits, row_bits=rb)
+    assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP, res
+    assert res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
+    assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL
