@@ -47,7 +47,6 @@ constexpr int kIoBytes = 512;       // stage room for one 128-vector input (fp32
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 4;            // rows per thread
-constexpr int kRpStride = 12;       // padded row stride of the row-maxima exchange (floats)
 constexpr unsigned kFull = 0xffffffffu;
 
 struct StageMeta {
@@ -85,7 +84,7 @@ struct DecodeArgs {
 
 // Shared memory besides the ring.
 struct Scratch {
-    float rp[DK * kRpStride];       // row maxima of |P| per panel
+    float rp[NPANEL * DK];          // row maxima of |P|: [panel][row] (conflict-free stores and loads)
     float4 wlo[DK];                 // per row {rho k, rho k, rho q, rho q}  (lanes 0..15)
     float4 whi[DK];                 // per row {rho q, rho q, rho k, rho k}  (lanes 16..31)
     float4 wrk[DK];                 // per row {rho, rho, k, k}
@@ -303,7 +302,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
 #pragma unroll
         for (int j = 3; j < PANEL - 1; j += 2) mx = absmax3(mx, T[m][j], T[m][j + 1]);
         mx = fmaxf(mx, fabsf(T[m][PANEL - 1]));
-        sc.rp[ix.row(m) * kRpStride + panel] = mx;
+        sc.rp[panel * DK + ix.row(m)] = mx;
     }
     if (__syncthreads_or(!ok)) return false;
 
@@ -311,9 +310,9 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     //      threads 128..255: the next state's row weights
     bool tiny = false;
     if (tid < DK) {
-        const float4 u = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride);
-        const float4 v = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride + 4);
-        const float mr = fmaxf(max3(u.x, u.y, u.z), max3(max3(u.w, v.x, v.y), v.z, v.w));
+        const float *rpt = sc.rp + tid;
+        const float mr = fmaxf(max3(rpt[0], rpt[DK], rpt[2 * DK]),
+                               max3(max3(rpt[3 * DK], rpt[4 * DK], rpt[5 * DK]), rpt[6 * DK], rpt[7 * DK]));
         float r;
         if constexpr (BITS == 0) {
             const int wdt = row_width(tid, n8, n4);
@@ -427,16 +426,16 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
 #pragma unroll
         for (int j = 3; j < PANEL - 1; j += 2) mx = absmax3(mx, T[m][j], T[m][j + 1]);
         mx = fmaxf(mx, fabsf(T[m][PANEL - 1]));
-        sc.rp[ix.row(m) * kRpStride + panel] = mx;
+        sc.rp[panel * DK + ix.row(m)] = mx;
     }
     if (__syncthreads_or(!ok)) return false;
 
     // ---- threads 0..127: r, 1/r and w r^2 of row tid (IEEE sqrt and divide; r is normal);
     //      threads 128..255: the next state's row weights
     if (tid < DK) {
-        const float4 u = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride);
-        const float4 v = *reinterpret_cast<const float4 *>(sc.rp + tid * kRpStride + 4);
-        const float mr = fmaxf(max3(u.x, u.y, u.z), max3(max3(u.w, v.x, v.y), v.z, v.w));
+        const float *rpt = sc.rp + tid;
+        const float mr = fmaxf(max3(rpt[0], rpt[DK], rpt[2 * DK]),
+                               max3(max3(rpt[3 * DK], rpt[4 * DK], rpt[5 * DK]), rpt[6 * DK], rpt[7 * DK]));
         const float w = a.impact[h * DK + tid];
         const float r = __fsqrt_rn(__fdiv_rn(mr, w));
         r_io[tid] = r;
@@ -647,7 +646,7 @@ struct ItemLoop {
     }
 };
 
-template <int GATE, typename TIn, bool IMPACT>
+template <int GATE, typename TIn, bool IMPACT, bool ROWS>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -707,8 +706,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     __syncthreads();
 
     int i = 0;
-    const bool done = L.template run<4>(i, end4) && L.template run<6>(i, end6) && L.template run<8>(i, end8) &&
-                      L.template run<0>(i, count);
+    // the class of heads with per-key-row widths is compiled only into the kernels of pools
+    // that have such heads
+    bool done = L.template run<4>(i, end4) && L.template run<6>(i, end6);
+    if constexpr (ROWS)
+        done = done && L.template run<8>(i, end8) && L.template run<0>(i, count);
+    else
+        done = done && L.template run<8>(i, count);
     const int lane = tid & 31;
     if (lane == 0) bulk_wait_all();
     if (tid == 0 && !done) {
@@ -849,19 +853,21 @@ size_t decode_smem_max()
 template <int GATE, typename TIn>
 cudaError_t configure_one(stepq_pool *p)
 {
-    auto kern = decode_kernel<GATE, TIn, false>;
-    auto kern_impact = decode_kernel<GATE, TIn, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(kern_impact, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
-    if (e != cudaSuccess) return e;
-    int per_sm = 0, per_sm_impact = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, p->decode_smem);
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_impact, kern_impact, kThreads, p->decode_smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1 || per_sm_impact < 1) return cudaErrorInvalidConfiguration;
-    p->decode_grid = (per_sm < per_sm_impact ? per_sm : per_sm_impact) * p->num_sms;
+    const void *kernels[4] = {reinterpret_cast<const void *>(decode_kernel<GATE, TIn, false, false>),
+                              reinterpret_cast<const void *>(decode_kernel<GATE, TIn, true, false>),
+                              reinterpret_cast<const void *>(decode_kernel<GATE, TIn, false, true>),
+                              reinterpret_cast<const void *>(decode_kernel<GATE, TIn, true, true>)};
+    int per_sm_min = 1 << 30;
+    for (const void *kern : kernels) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(decode_smem_max()));
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, p->decode_smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < per_sm_min) per_sm_min = per_sm;
+    }
+    if (per_sm_min < 1) return cudaErrorInvalidConfiguration;
+    p->decode_grid = per_sm_min * p->num_sms;
     return cudaSuccess;
 }
 
@@ -872,6 +878,22 @@ cudaError_t upload_tables()
     for (int b = 0; b < 3; ++b)
         for (int p = 0; p < PANEL; ++p) h[b][p] = 1.0f / pos_scale(widths[b], p);
     return cudaMemcpyToSymbol(kInvPos, h, sizeof(h));
+}
+
+template <int GATE, typename TIn>
+void launch_variant(bool impact, bool rows, int grid, size_t smem, cudaStream_t stream, const DecodeArgs &a)
+{
+    if (impact) {
+        if (rows)
+            decode_kernel<GATE, TIn, true, true><<<grid, kThreads, smem, stream>>>(a);
+        else
+            decode_kernel<GATE, TIn, true, false><<<grid, kThreads, smem, stream>>>(a);
+    } else {
+        if (rows)
+            decode_kernel<GATE, TIn, false, true><<<grid, kThreads, smem, stream>>>(a);
+        else
+            decode_kernel<GATE, TIn, false, false><<<grid, kThreads, smem, stream>>>(a);
+    }
 }
 
 void count_widths(const uint8_t *bits, int H, DecodeArgs &a)
@@ -937,28 +959,17 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
         a.step_b = grid % n;
         a.step_h = grid / n;
         const size_t sm = p->decode_smem;
-        if (a.impact) {
-            if (p->gate_mode == STEPQ_GATE_GDN) {
-                if (p->in_dtype == STEPQ_DTYPE_BF16)
-                    decode_kernel<STEPQ_GATE_GDN, uint16_t, true><<<grid, kThreads, sm, stream>>>(a);
-                else
-                    decode_kernel<STEPQ_GATE_GDN, float, true><<<grid, kThreads, sm, stream>>>(a);
-            } else {
-                if (p->in_dtype == STEPQ_DTYPE_BF16)
-                    decode_kernel<STEPQ_GATE_KDA, uint16_t, true><<<grid, kThreads, sm, stream>>>(a);
-                else
-                    decode_kernel<STEPQ_GATE_KDA, float, true><<<grid, kThreads, sm, stream>>>(a);
-            }
-        } else if (p->gate_mode == STEPQ_GATE_GDN) {
+        const bool rows = p->d_perm != nullptr;
+        if (p->gate_mode == STEPQ_GATE_GDN) {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                decode_kernel<STEPQ_GATE_GDN, uint16_t, false><<<grid, kThreads, sm, stream>>>(a);
+                launch_variant<STEPQ_GATE_GDN, uint16_t>(a.impact != nullptr, rows, grid, sm, stream, a);
             else
-                decode_kernel<STEPQ_GATE_GDN, float, false><<<grid, kThreads, sm, stream>>>(a);
+                launch_variant<STEPQ_GATE_GDN, float>(a.impact != nullptr, rows, grid, sm, stream, a);
         } else {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                decode_kernel<STEPQ_GATE_KDA, uint16_t, false><<<grid, kThreads, sm, stream>>>(a);
+                launch_variant<STEPQ_GATE_KDA, uint16_t>(a.impact != nullptr, rows, grid, sm, stream, a);
             else
-                decode_kernel<STEPQ_GATE_KDA, float, false><<<grid, kThreads, sm, stream>>>(a);
+                launch_variant<STEPQ_GATE_KDA, float>(a.impact != nullptr, rows, grid, sm, stream, a);
         }
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -1028,13 +1039,13 @@ cudaError_t noalloc_setup(int dev, NoallocDevice **out)
         e = upload_tables();
         if (e != cudaSuccess) return e;
         const int smem = int(decode_smem_max());
-        e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, float, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, uint16_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_GDN, uint16_t, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, float, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, uint16_t, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            e = cudaFuncSetAttribute(decode_kernel<STEPQ_GATE_KDA, uint16_t, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         d.scratch = static_cast<uint8_t *>(ptr);
         d.ready = true;
@@ -1048,7 +1059,7 @@ cudaError_t noalloc_launch(const DecodeArgs &a0, int num_sms, size_t smem, cudaS
 {
     DecodeArgs a = a0;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<GATE, TIn, false>, kThreads, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<GATE, TIn, false, false>, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long total = (long long)a.n * a.H;
@@ -1056,7 +1067,7 @@ cudaError_t noalloc_launch(const DecodeArgs &a0, int num_sms, size_t smem, cudaS
     const int grid = int(total < cap ? total : cap);
     a.step_b = grid % a.n;
     a.step_h = grid / a.n;
-    decode_kernel<GATE, TIn, false><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<GATE, TIn, false, false><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
