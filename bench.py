@@ -187,8 +187,29 @@ def cpu_baseline(w, bits, seconds: float):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": steps * len(sl) * w.H / el, "unit": UNIT, "cores": O.default_threads(), "kind": "oracle",
-            "sample": "%d requests x %d heads x %d decode steps of %s (%.1f s)" % (len(sl), w.H, steps, w.name, el)}
+    value = steps * len(sl) * w.H / el
+    # the same oracle on one core, over a shorter bounded sample
+    one = 0
+    t1 = time.perf_counter()
+    while True:
+        pool.decode_step(sl[:2], **{k: v[:2] for k, v in xs[one % len(xs)].items()}, nthreads=1)
+        one += 1
+        el1 = time.perf_counter() - t1
+        if el1 >= seconds / 3:
+            break
+    return {"value": value, "unit": UNIT, "cores": O.default_threads(), "kind": "oracle",
+            "sample": "%d requests x %d heads x %d decode steps of %s (%.1f s)" % (len(sl), w.H, steps, w.name, el),
+            "one_core_value": one * 2 * w.H / el1, "host_cpus": os.cpu_count(), "cpu_model": _cpu_model()}
+
+
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args):
@@ -409,6 +430,36 @@ def main():
     peak, peak_kind = peaks()
     achieved = alg_bytes / avg_kernel_s / 1e9
 
+    # ---- the same step as a CUDA graph of T = 16 launches, replayed: median over 12 replays
+    graph_us = None
+    try:
+        T = 16
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for t in range(T):
+                    x = sets[t % nsets]
+                    pool.decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y, side)
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize()
+        reps = []
+        for _ in range(12):
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            g.replay()
+            g1.record(stream)
+            torch.cuda.synchronize()
+            reps.append(g0.elapsed_time(g1) * 1e3 / T)
+        graph_us = statistics.median(reps)
+        del g
+    except Exception as exc:                      # graph capture is informational only
+        graph_us = "unavailable: %s" % type(exc).__name__
+    if pool.get_error() != 0:
+        raise RuntimeError("device flag set in the graph leg")
+
     # ---- end-to-end leg: host inputs in pinned memory, H2D + decode + D2H of y every step
     host = []
     for x in host_sets[:E2E_HOST_SETS]:
@@ -467,6 +518,7 @@ def main():
                          "kernel": "decode_kernel", "avg_kernel_us": avg_kernel_s * 1e6},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
+            "graph_us_per_step": graph_us,
             "gpu_launches": args.steps * (2 if int(np.sum(bits == 16)) else 1),   # + pivot kernel
             "clocks": clocks,
             "cpu_baseline": base,
