@@ -194,6 +194,13 @@ STEPQ_API int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *st
  * non-positive or non-finite score. */
 STEPQ_API int stepq_pool_set_impact(stepq_pool *pool, const float *impact);
 
+/* Health check of the kernels' failure path: a one-warp kernel waits on a shared-memory
+ * barrier that nothing completes (no copy in flight), with the same bounded wait as the
+ * decode kernel but a short poll limit, then raises STEPQ_FLAG_TIMEOUT and exits.  flag_out
+ * (HOST) receives the flag bits: STEPQ_FLAG_TIMEOUT when the path works.  The context stays
+ * usable.  Synchronizes `stream`. */
+STEPQ_API int stepq_check_wait_timeout(int32_t *flag_out, stepq_stream stream);
+
 /* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
  * Synchronizes the device. */
 STEPQ_API int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out);

@@ -313,6 +313,24 @@ int stepq_pool_set_impact(stepq_pool *pool, const float *impact)
     return status_of(e);
 }
 
+int stepq_check_wait_timeout(int32_t *flag_out, stepq_stream stream)
+{
+    if (!flag_out) return STEPQ_INVALID_ARG;
+    int *d_flag = nullptr;
+    cudaError_t e = cudaMalloc(&d_flag, sizeof(int));
+    if (e != cudaSuccess) return status_of(e);
+    e = cudaMemsetAsync(d_flag, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = stepq::launch_wait_check(d_flag, stream);
+    int h = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&h, d_flag, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    const cudaError_t ef = cudaFree(d_flag);
+    if (e == cudaSuccess) e = ef;
+    if (e != cudaSuccess) return status_of(e);
+    *flag_out = h;
+    return STEPQ_OK;
+}
+
 int stepq_pool_get_error(stepq_pool *pool, int32_t *flag_out)
 {
     if (!pool || !flag_out) return STEPQ_INVALID_ARG;

@@ -46,6 +46,7 @@ cudaError_t decode_configure(stepq_pool *p);
 cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, const void *q,
                           const void *k, const void *v, const void *alpha, const void *beta,
                           float *y, cudaStream_t stream);
+cudaError_t launch_wait_check(int *flag, cudaStream_t stream);
 cudaError_t launch_load_fp32(const stepq_pool *p, const int32_t *slot_ids, int n, const float *S,
                              cudaStream_t stream);
 cudaError_t launch_dump_fp32(const stepq_pool *p, const int32_t *slot_ids, int n, float *S,

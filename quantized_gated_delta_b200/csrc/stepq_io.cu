@@ -362,6 +362,27 @@ __global__ void copy_slots_kernel(const IoArgs a, const uint8_t *src, uint8_t *d
 }
 
 // ------------------------------------------------------------------------------------------
+// The bounded-wait path of the kernels, on its own: one warp waits on a shared-memory
+// mbarrier that nothing completes (no copy is in flight), gives up after a short poll limit,
+// raises the timeout bit of the flag and returns -- the same steps a decode CTA takes when a
+// stage never arrives, with a limit short enough for a health check.
+// ------------------------------------------------------------------------------------------
+__global__ void wait_check_kernel(int *flag)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbarrier_init();
+    }
+    __syncwarp();
+    const bool ok = mbar_wait_bounded<1024>(&bar, 0u);
+    if (threadIdx.x == 0) {
+        if (!ok) atomicOr(flag, STEPQ_FLAG_TIMEOUT);
+        mbar_arrive(&bar);                         // leave the barrier in a completed phase
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Launchers
 // ------------------------------------------------------------------------------------------
 namespace {
@@ -386,6 +407,12 @@ IoArgs io_args(const stepq_pool *p, const int32_t *slot_ids)
 }
 
 }  // namespace
+
+cudaError_t launch_wait_check(int *flag, cudaStream_t stream)
+{
+    wait_check_kernel<<<1, 32, 0, stream>>>(flag);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_load_fp32(const stepq_pool *p, const int32_t *slot_ids, int n, const float *S,
                              cudaStream_t stream)

@@ -29,6 +29,7 @@ EXPORTED = [
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
     "stepq_allocate_bits_pivots", "stepq_pool_set_impact", "stepq_pool_create_rows",
+    "stepq_check_wait_timeout",
 ]
 
 
@@ -70,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_allocate_bits": [P, P, I, P, I, ctypes.c_double, P],
         "stepq_allocate_bits_pivots": [P, P, I, P, I, ctypes.c_double, I, P],
         "stepq_pool_set_impact": [P, P],
+        "stepq_check_wait_timeout": [ctypes.POINTER(I), P],
         "stepq_pool_create_rows": [ctypes.POINTER(stepq_pool_desc), P, ctypes.POINTER(P)],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
@@ -201,6 +203,14 @@ def stepq_pool_set_impact(pool: int, impact=None):
         return
     w = np.ascontiguousarray(impact, dtype=np.float32)
     _check(load_library().stepq_pool_set_impact(pool, w.ctypes.data), "stepq_pool_set_impact")
+
+
+def stepq_check_wait_timeout(stream=None) -> int:
+    """Run the kernels' bounded-wait failure path on a barrier nothing completes; returns the
+    flag bits it raised (STEPQ_FLAG_TIMEOUT when the path works)."""
+    f = ctypes.c_int32()
+    _check(load_library().stepq_check_wait_timeout(ctypes.byref(f), _stream(stream)), "stepq_check_wait_timeout")
+    return f.value
 
 
 def stepq_pool_get_error(pool: int) -> int:

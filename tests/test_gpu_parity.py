@@ -329,6 +329,30 @@ def test_zero_requests_and_invalid_arguments(S):
     assert gp.get_error() == 0
 
 
+def test_bounded_wait_timeout_reports_and_context_survives(S):
+    """The kernels' failure path: a bounded wait on a barrier that nothing completes gives up,
+    raises the timeout flag for the host, and the context keeps working (a decode step right
+    after it matches the same step on a fresh pool)."""
+    rng = np.random.default_rng(11)
+    bits, n, H = [4, 8], 3, 2
+    states = random_states(rng, n, H)
+    op = O.OraclePool(n, bits, H)
+    op.load_fp32(np.arange(n, dtype=np.int32), states)
+    per_req = op.slot_bytes(np.arange(n))
+    x = dict(q=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+             k=np.stack([[unit(rng, 128) for _ in range(H)] for _ in range(n)]),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.8, 1, (n, H)).astype(f32), beta=rng.uniform(0, 1, (n, H)).astype(f32))
+    ids = np.arange(n, dtype=np.int32)
+    y0, s0, e0 = _run_gpu(S, bits, H, 0, S.STEPQ_DTYPE_F32, x, per_req, ids, n)
+    for _ in range(2):
+        assert S.stepq_check_wait_timeout() == S.STEPQ_FLAG_TIMEOUT
+    torch.cuda.synchronize()
+    y1, s1, e1 = _run_gpu(S, bits, H, 0, S.STEPQ_DTYPE_F32, x, per_req, ids, n)
+    assert e0 == e1 == 0
+    assert np.array_equal(y0, y1) and np.array_equal(s0, s1)
+
+
 # --------------------------------------------------------------------------- workload parity
 
 CASES = [
