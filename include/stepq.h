@@ -156,6 +156,30 @@ STEPQ_API int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32
                       const void *k, const void *v, const void *alpha, const void *beta, float *y,
                       stepq_stream stream);
 
+/* The decode step of stepq_decode_step with every per-step buffer in HOST memory: the call
+ * copies slot_ids and the inputs into a device staging buffer owned by the pool, runs the
+ * step, and copies y back.  The paper has no counterpart to this entry point; it is the
+ * path of a caller whose tokens arrive in host memory.  All of it is asynchronous:
+ *   slot_ids [n] int32, q, k, v, alpha, beta   HOST, layouts and dtypes as for stepq_decode_step
+ *   y        HOST [n, H, d_v] float32, written when the call's copy-out runs
+ * The pool keeps two staging buffers and uses them in turn; the inputs are copied on a
+ * copy-in stream of the pool, the step runs on `stream`, and y is copied on a copy-out stream
+ * of the pool, chained by events, so the copies of consecutive calls overlap the steps of
+ * their neighbours.  Host buffers must stay valid and unchanged (inputs), or unread (y),
+ * until the call's copies are done: after stepq_pool_host_wait(pool, s) and a
+ * synchronization of s.  Page-locked host memory lets the copies run asynchronously;
+ * pageable memory works, with copies that hold up the calling thread.  The first call, and a
+ * call with more requests than any before it, allocates the staging buffers (a regrowth first
+ * waits for the copies of the earlier calls).  A pool must not be used from several host
+ * threads at once.  Errors: as for stepq_decode_step; argument checks come before any copy. */
+STEPQ_API int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q,
+                                     const void *k, const void *v, const void *alpha, const void *beta, float *y,
+                                     stepq_stream stream);
+
+/* Makes `stream` wait for every copy that stepq_decode_step_host calls on this pool have
+ * enqueued, y included.  Enqueues only; synchronize `stream` to wait on the host. */
+STEPQ_API int stepq_pool_host_wait(stepq_pool *pool, stepq_stream stream);
+
 /* The decode step of stepq_decode_step for callers that cannot allocate device memory.
  * The paper has no counterpart to this entry point.  Some callers may not call cudaMalloc:
  * code running inside a serving engine or framework that owns all device memory through

@@ -54,7 +54,76 @@ void free_pool(stepq_pool *p)
     cudaFree(p->d_rn4);
     cudaFree(p->d_rpb);
     cudaFree(p->d_perm);
+    for (int b = 0; b < 2; ++b) {
+        cudaFree(p->d_host_stage[b]);
+        if (p->ev_in[b]) cudaEventDestroy(p->ev_in[b]);
+        if (p->ev_step[b]) cudaEventDestroy(p->ev_step[b]);
+        if (p->ev_out[b]) cudaEventDestroy(p->ev_out[b]);
+    }
+    if (p->s_in) cudaStreamDestroy(p->s_in);
+    if (p->s_out) cudaStreamDestroy(p->s_out);
     delete p;
+}
+
+// ---- host-buffer decode: byte offsets of one call's inputs and output in a staging buffer
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct HostLayout {
+    size_t slots, q, k, v, alpha, beta, y, total;
+    size_t qk_bytes, v_bytes, alpha_bytes, beta_bytes, y_bytes;
+};
+
+HostLayout host_layout(const stepq_pool *p, int n)
+{
+    const size_t esz = p->in_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
+    HostLayout L;
+    L.qk_bytes = size_t(n) * p->Hk * 128 * esz;
+    L.v_bytes = size_t(n) * p->H * 128 * esz;
+    L.alpha_bytes = size_t(n) * p->H * (p->gate_mode == STEPQ_GATE_KDA ? 128 : 1) * esz;
+    L.beta_bytes = size_t(n) * p->H * esz;
+    L.y_bytes = size_t(n) * p->H * 128 * 4;
+    size_t o = 0;
+    L.slots = o; o += round256(size_t(n) * 4);
+    L.q = o; o += round256(L.qk_bytes);
+    L.k = o; o += round256(L.qk_bytes);
+    L.v = o; o += round256(L.v_bytes);
+    L.alpha = o; o += round256(L.alpha_bytes);
+    L.beta = o; o += round256(L.beta_bytes);
+    L.y = o; o += round256(L.y_bytes);
+    L.total = o;
+    return L;
+}
+
+// Streams, events and staging buffers of the host-buffer path: created on the first call,
+// regrown (once every earlier use has finished) when a call needs more room.
+int host_prepare(stepq_pool *p, size_t bytes)
+{
+    cudaError_t e = cudaSuccess;
+    if (!p->s_in) {
+        e = cudaStreamCreateWithFlags(&p->s_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->s_out, cudaStreamNonBlocking);
+        for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+            e = cudaEventCreateWithFlags(&p->ev_in[b], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_step[b], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_out[b], cudaEventDisableTiming);
+        }
+        if (e != cudaSuccess) return status_of(e);
+    }
+    if (bytes <= p->host_stage_cap) return STEPQ_OK;
+    // every earlier use of a staging buffer ends with its copy-out
+    for (int b = 0; b < 2 && e == cudaSuccess; ++b) e = cudaEventSynchronize(p->ev_out[b]);
+    if (e != cudaSuccess) return status_of(e);
+    for (int b = 0; b < 2; ++b) {
+        cudaFree(p->d_host_stage[b]);
+        p->d_host_stage[b] = nullptr;
+    }
+    p->host_stage_cap = 0;
+    for (int b = 0; b < 2; ++b) {
+        e = cudaMalloc(&p->d_host_stage[b], bytes);
+        if (e != cudaSuccess) return status_of(e);
+    }
+    p->host_stage_cap = bytes;
+    return STEPQ_OK;
 }
 
 }  // namespace
@@ -279,6 +348,55 @@ int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, cons
     if (pool->gate_mode == STEPQ_GATE_KDA ? !aligned16(alpha) : !aligned_to(alpha, esz)) return STEPQ_INVALID_ARG;
     if (!aligned_to(beta, esz)) return STEPQ_INVALID_ARG;
     return status_of(stepq::launch_decode(pool, slot_ids, n, q, k, v, alpha, beta, y, stream));
+}
+
+int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q, const void *k,
+                           const void *v, const void *alpha, const void *beta, float *y, stepq_stream stream)
+{
+    if (!pool || n < 0 || n > pool->num_slots || n > 65535) return STEPQ_INVALID_ARG;
+    int st = check_device(pool);
+    if (st != STEPQ_OK) return st;
+    if (n == 0) return STEPQ_OK;
+    if (!slot_ids || !q || !k || !v || !alpha || !beta || !y) return STEPQ_INVALID_ARG;
+    const HostLayout L = host_layout(pool, n);
+    st = host_prepare(pool, L.total);
+    if (st != STEPQ_OK) return st;
+    const int b = int(pool->host_calls & 1);
+    uint8_t *d = pool->d_host_stage[b];
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+    // copy-in, once the step that last read this staging buffer is done
+    cudaError_t e = cudaStreamWaitEvent(pool->s_in, pool->ev_step[b], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.slots, slot_ids, size_t(n) * 4, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.q, q, L.qk_bytes, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.k, k, L.qk_bytes, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.v, v, L.v_bytes, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.alpha, alpha, L.alpha_bytes, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.beta, beta, L.beta_bytes, h2d, pool->s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(pool->ev_in[b], pool->s_in);
+    // the step on the caller's stream, once its inputs are in and the copy-out that last read
+    // this buffer's y is done
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, pool->ev_in[b], 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, pool->ev_out[b], 0);
+    if (e == cudaSuccess)
+        e = stepq::launch_decode(pool, reinterpret_cast<const int32_t *>(d + L.slots), n, d + L.q, d + L.k, d + L.v,
+                                 d + L.alpha, d + L.beta, reinterpret_cast<float *>(d + L.y), stream);
+    if (e == cudaSuccess) e = cudaEventRecord(pool->ev_step[b], stream);
+    // copy-out of y
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(pool->s_out, pool->ev_step[b], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(y, d + L.y, L.y_bytes, cudaMemcpyDeviceToHost, pool->s_out);
+    if (e == cudaSuccess) e = cudaEventRecord(pool->ev_out[b], pool->s_out);
+    ++pool->host_calls;
+    return status_of(e);
+}
+
+int stepq_pool_host_wait(stepq_pool *pool, stepq_stream stream)
+{
+    if (!pool) return STEPQ_INVALID_ARG;
+    int st = check_device(pool);
+    if (st != STEPQ_OK || !pool->s_in) return st;
+    cudaError_t e = cudaSuccess;
+    for (int b = 0; b < 2 && e == cudaSuccess; ++b) e = cudaStreamWaitEvent(stream, pool->ev_out[b], 0);
+    return status_of(e);
 }
 
 int stepq_pool_set_impact(stepq_pool *pool, const float *impact)

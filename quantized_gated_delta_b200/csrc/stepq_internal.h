@@ -35,6 +35,14 @@ struct stepq_pool {
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel
     int stage_bytes = 0;
     int blk_cap = 0;
+    // host-buffer decode (stepq_decode_step_host): two device staging buffers used in turn,
+    // the copy-in and copy-out streams, and the events that chain copy-in -> step -> copy-out;
+    // created on first use
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_step[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
+    uint8_t *d_host_stage[2] = {nullptr, nullptr};
+    size_t host_stage_cap = 0;          // bytes of each staging buffer
+    long long host_calls = 0;
 };
 
 namespace stepq {

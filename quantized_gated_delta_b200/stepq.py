@@ -29,7 +29,7 @@ EXPORTED = [
     "stepq_pool_dump_packed", "stepq_decode_step", "stepq_pool_get_error",
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
     "stepq_allocate_bits_pivots", "stepq_pool_set_impact", "stepq_pool_create_rows",
-    "stepq_check_wait_timeout",
+    "stepq_check_wait_timeout", "stepq_decode_step_host", "stepq_pool_host_wait",
 ]
 
 
@@ -72,6 +72,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_allocate_bits_pivots": [P, P, I, P, I, ctypes.c_double, I, P],
         "stepq_pool_set_impact": [P, P],
         "stepq_check_wait_timeout": [ctypes.POINTER(I), P],
+        "stepq_decode_step_host": [P, P, I, P, P, P, P, P, P, P],
+        "stepq_pool_host_wait": [P, P],
         "stepq_pool_create_rows": [ctypes.POINTER(stepq_pool_desc), P, ctypes.POINTER(P)],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
     }
@@ -180,6 +182,25 @@ def stepq_decode_step(pool: int, slot_ids, q, k, v, alpha, beta, y, stream=None)
         _dev(alpha, "alpha"), _dev(beta, "beta"), _dev(y, "y"), _stream(stream)), "stepq_decode_step")
 
 
+def _host(t, name):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous host tensor" % name)
+    return t.data_ptr()
+
+
+def stepq_decode_step_host(pool: int, slot_ids, q, k, v, alpha, beta, y, stream=None):
+    """Decode step with every per-step buffer in host memory (pinned for overlapped copies):
+    copy-in, step and copy-out are asynchronous; ``stepq_pool_host_wait`` orders a stream
+    after the copies."""
+    _check(load_library().stepq_decode_step_host(
+        pool, _host(slot_ids, "slot_ids"), slot_ids.numel(), _host(q, "q"), _host(k, "k"), _host(v, "v"),
+        _host(alpha, "alpha"), _host(beta, "beta"), _host(y, "y"), _stream(stream)), "stepq_decode_step_host")
+
+
+def stepq_pool_host_wait(pool: int, stream=None):
+    _check(load_library().stepq_pool_host_wait(pool, _stream(stream)), "stepq_pool_host_wait")
+
+
 def stepq_decode_step_noalloc(num_slots: int, head_bits, num_key_heads: int, gate_mode: int, in_dtype: int,
                               state, slot_ids, q, k, v, alpha, beta, y, flag_out=None, stream=None):
     """Decode step on a caller-owned packed state buffer; the library allocates nothing.
@@ -277,6 +298,12 @@ class Pool:
 
     def decode_step(self, slot_ids, q, k, v, alpha, beta, y, stream=None):
         stepq_decode_step(self.handle, slot_ids, q, k, v, alpha, beta, y, stream)
+
+    def decode_step_host(self, slot_ids, q, k, v, alpha, beta, y, stream=None):
+        stepq_decode_step_host(self.handle, slot_ids, q, k, v, alpha, beta, y, stream)
+
+    def host_wait(self, stream=None):
+        stepq_pool_host_wait(self.handle, stream)
 
     def load_fp32(self, slot_ids, S, stream=None):
         stepq_pool_load_fp32(self.handle, slot_ids, S, stream)

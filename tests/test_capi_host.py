@@ -66,6 +66,8 @@ def test_descriptor_validation_before_device(S):
     assert lib.stepq_pool_destroy(None) == 0
     assert lib.stepq_pool_bytes(None, None, None) == -1
     assert lib.stepq_decode_step(None, None, 0, None, None, None, None, None, None, None) == -1
+    assert lib.stepq_decode_step_host(None, None, 0, None, None, None, None, None, None, None) == -1
+    assert lib.stepq_pool_host_wait(None, None) == -1
 
 
 @pytest.mark.parametrize("N", [1, 3, 6, 8])

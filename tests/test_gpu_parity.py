@@ -329,6 +329,51 @@ def test_zero_requests_and_invalid_arguments(S):
     assert gp.get_error() == 0
 
 
+def test_host_buffer_steps_match_device_steps(S):
+    """stepq_decode_step_host (slot ids, inputs and y in host memory; copy-in, step and
+    copy-out of consecutive calls overlapped through two staging buffers) gives outputs and
+    states bit-identical to stepq_decode_step on device buffers, call after call: six calls
+    enqueued back to back on pinned buffers, then one on pageable buffers, then a larger
+    batch that regrows the staging buffers."""
+    rng = np.random.default_rng(5)
+    bits, H, Hk, num_slots = [4, 6, 8, 6], 4, 2, 12
+    ids_all = np.array([6, 1, 3, 0, 5, 9, 11, 2], np.int32)
+    S0 = torch.from_numpy(random_states(rng, len(ids_all), H)).cuda()
+    pools = [S.Pool(num_slots, bits, Hk, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_BF16) for _ in range(2)]
+    for gp in pools:
+        gp.load_fp32(slots_t(ids_all), S0)
+
+    def inputs(n):
+        x = dict(q=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
+                 k=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
+                 v=rng.standard_normal((n, H, 128)).astype(f32),
+                 alpha=rng.uniform(0.8, 1, (n, H)).astype(f32), beta=rng.uniform(0, 1, (n, H)).astype(f32))
+        return {key: torch.from_numpy(W.to_bf16_bits(val).view(np.int16)) for key, val in x.items()}
+
+    plan = [(5, True)] * 6 + [(5, False), (8, True)]
+    steps = [(ids_all[:n], inputs(n), pinned) for n, pinned in plan]
+    y_dev = []
+    for ids, x, _ in steps:
+        y = torch.empty((len(ids), H, 128), device="cuda")
+        pools[0].decode_step(slots_t(ids), *[x[key].cuda() for key in ("q", "k", "v", "alpha", "beta")], y)
+        y_dev.append(y.cpu().numpy())
+    y_host = []
+    for ids, x, pinned in steps:
+        hx = {key: (val.pin_memory() if pinned else val.clone()) for key, val in x.items()}
+        hs = torch.from_numpy(ids.copy())
+        yh = torch.full((len(ids), H, 128), float("nan"))
+        if pinned:
+            hs, yh = hs.pin_memory(), yh.pin_memory()
+        pools[1].decode_step_host(hs, hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], yh)
+        y_host.append((yh, hx, hs))                 # keep the host buffers alive until the wait
+    pools[1].host_wait()
+    torch.cuda.synchronize()
+    for t, (yd, (yh, _, _)) in enumerate(zip(y_dev, y_host)):
+        assert np.array_equal(yd, yh.numpy()), "call %d" % t
+    assert np.array_equal(dump_bytes(pools[0], ids_all), dump_bytes(pools[1], ids_all))
+    assert pools[0].get_error() == 0 and pools[1].get_error() == 0
+
+
 def test_bounded_wait_timeout_reports_and_context_survives(S):
     """The kernels' failure path: a bounded wait on a barrier that nothing completes gives up,
     raises the timeout flag for the host, and the context keeps working (a decode step right
