@@ -33,6 +33,7 @@
 // from the stage (warp 0 also r).  Each state is read from HBM once and written once.
 #include <cfloat>
 #include <cstdint>
+#include <type_traits>
 #include <cuda_fp16.h>
 
 #include "stepq_internal.h"
@@ -48,6 +49,14 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRows = 4;            // rows per thread
 constexpr unsigned kFull = 0xffffffffu;
+// Stage of the ring: room for the largest quantized head block (8-bit codes + r + c; a head
+// with per-key-row widths is never larger), then q, k, v and, for KDA, the gate vector.
+constexpr int kBlkCap = block_bytes(8);
+template <int GATE>
+__host__ __device__ constexpr int stage_bytes_of()
+{
+    return (kBlkCap + (GATE == STEPQ_GATE_KDA ? 4 : 3) * kIoBytes + 127) / 128 * 128;
+}
 
 struct StageMeta {
     long long dst;                  // byte offset of the head block in the pool
@@ -79,7 +88,6 @@ struct DecodeArgs {
     const void *q, *k, *v, *alpha, *beta;
     float *y;
     int *flag;
-    int blk_cap, stage_bytes;
 };
 
 // Shared memory besides the ring.
@@ -119,16 +127,17 @@ struct Cursor {
 
 // Per-row weights of a state held in a stage, built by thread t (128 <= t < 256) for row
 // t - 128, and the share of k.q of warps 4..7.
-template <int GATE, typename TIn>
+template <int GATE, typename TIn, bool ROWS>
 __device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs &a, int bits, int head,
                                           float alpha_s, Scratch &sc, int t)
 {
     const int i = t - 128;                          // stored row (the key row unless bits == 0)
-    const float *r = reinterpret_cast<const float *>(stage + (bits ? codes_bytes(bits) : 8 * a.row_pb[head]));
-    const int key = bits ? i : int(a.row_perm[head * DK + i]);
-    const TIn *qs = reinterpret_cast<const TIn *>(stage + a.blk_cap);
-    const TIn *ks = reinterpret_cast<const TIn *>(stage + a.blk_cap + kIoBytes);
-    const TIn *as = reinterpret_cast<const TIn *>(stage + a.blk_cap + 3 * kIoBytes);
+    const bool rows = ROWS && bits == 0;            // heads with per-key-row widths exist only in ROWS pools
+    const float *r = reinterpret_cast<const float *>(stage + (rows ? 8 * a.row_pb[head] : codes_bytes(bits)));
+    const int key = rows ? int(a.row_perm[head * DK + i]) : i;
+    const TIn *qs = reinterpret_cast<const TIn *>(stage + kBlkCap);
+    const TIn *ks = reinterpret_cast<const TIn *>(stage + kBlkCap + kIoBytes);
+    const TIn *as = reinterpret_cast<const TIn *>(stage + kBlkCap + 3 * kIoBytes);
     const float al = (GATE == STEPQ_GATE_KDA) ? to_f32(as[key]) : alpha_s;
     const float rho = al * r[i];
     const float k = to_f32(ks[key]);
@@ -146,18 +155,18 @@ __device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs
 // One state: the register tile through the row-maxima exchange, the row finalization /
 // next row table, then quantization, packing and the per-warp stores.  Returns false on
 // every thread when some thread saw a failed wait.
-template <int GATE, typename TIn, int BITS>
+template <int GATE, typename TIn, int BITS, bool ROWS>
 __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *stages, int i, bool has_next,
                                              const DecodeArgs &a, Scratch &sc, const TileIdx<4> &ix, int tid, int h,
                                              float cprime, TIn alpha_next_raw, bool ok, float *r_io, float *c_io,
                                              uint8_t *codes);
 
-template <int GATE, typename TIn, int BITS, bool IMPACT>
+template <int GATE, typename TIn, int BITS, bool IMPACT, bool ROWS>
 __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_next, const DecodeArgs &a, Scratch &sc,
                                             const TileIdx<4> &ix, int tid, long long bh, float beta, float kq,
                                             TIn alpha_next_raw, bool ok)
 {
-    uint8_t *stage = stages + (i % kStages) * a.stage_bytes;
+    uint8_t *stage = stages + (i % kStages) * stage_bytes_of<GATE>();
     // BITS == 0: per-key-row widths (rows stored 8-bit, 4-bit, 6-bit; codes unscaled)
     constexpr int QM = BITS ? qmax_of(BITS) : 1;
     constexpr float MAG = kTwo23 + float(1 << ((BITS ? BITS : 1) - 1));
@@ -178,7 +187,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     uint8_t *codes = stage;
     float *r_io = reinterpret_cast<float *>(stage + cbytes);
     float *c_io = r_io + DK;
-    const TIn *vs = reinterpret_cast<const TIn *>(stage + a.blk_cap + 2 * kIoBytes);
+    const TIn *vs = reinterpret_cast<const TIn *>(stage + kBlkCap + 2 * kIoBytes);
 
     // ---- codes of the thread's 4 rows x 16 columns (times their position scale), exact floats
     float T[kRows][PANEL];
@@ -230,8 +239,9 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
             s1 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].x, w[m].y), s1);
             s2 = ffma2(make_float2(T[m][j], T[m][j + 1]), make_float2(w[m].z, w[m].w), s2);
         }
-        A[j] = s1.x + __shfl_xor_sync(kFull, s2.x, 16);
-        A[j + 1] = s1.y + __shfl_xor_sync(kFull, s2.y, 16);
+        const float2 t = fadd2(s1, make_float2(__shfl_xor_sync(kFull, s2.x, 16), __shfl_xor_sync(kFull, s2.y, 16)));
+        A[j] = t.x;
+        A[j + 1] = t.y;
     }
     reduce_scatter<PANEL, 4, 8, false>(A, lane);
 
@@ -262,7 +272,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         }
     }
     if constexpr (IMPACT && BITS != 0)          // heads with per-row widths keep the clip-free fit
-        return refit_impact<GATE, TIn, BITS>(T, stages, i, has_next, a, sc, ix, tid, int(bh % a.H), cprime,
+        return refit_impact<GATE, TIn, BITS, ROWS>(T, stages, i, has_next, a, sc, ix, tid, int(bh % a.H), cprime,
                                              alpha_next_raw, ok, r_io, c_io, codes);
     // column maxima: over the thread's rows, then a warp-wide max per column; the 16
     // results go through shared memory (the d' buffer, already read) to the column lanes
@@ -328,53 +338,61 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         r_io[tid] = r;
         tiny = r > 0.0f && r < FLT_MIN;
     } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
-        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
+        row_table<GATE, TIn, ROWS>(stages + ((i + 1) % kStages) * stage_bytes_of<GATE>(), a, sc.meta[(i + 1) % kStages].bits,
                              sc.meta[(i + 1) % kStages].head, to_f32(alpha_next_raw), sc, tid);
     }
     const bool any_tiny = __syncthreads_or(tiny);
 
     // ---- codes = round-half-even(P_ij / r_i): fma(P, 1/r, 2^23 + 2^(b-1)) rounds to the
-    // nearest integer, ties to even, leaving the offset-binary code in the low mantissa bits
+    // nearest integer, ties to even, leaving the offset-binary code in the low mantissa bits.
+    // The block-uniform any_tiny picks one of two copies of the loop, so the common copy has
+    // no per-row test.
+    auto quantize_pack = [&](auto tiny_rows) {
 #pragma unroll
-    for (int m = 0; m < kRows; ++m) {
-        const int row = ix.row(m);
-        float2 ir, mag2 = make_float2(MAG, MAG);
-        if constexpr (BITS == 0) {
-            const float4 f = sc.fit[row];
-            ir = make_float2(f.x, f.y);
-            mag2 = make_float2(f.z, f.w);
-        } else {
-            ir = sc.ir[row];
-        }
-        uint32_t u[PANEL];
+        for (int m = 0; m < kRows; ++m) {
+            const int row = ix.row(m);
+            float2 ir, mag2 = make_float2(MAG, MAG);
+            if constexpr (BITS == 0) {
+                const float4 f = sc.fit[row];
+                ir = make_float2(f.x, f.y);
+                mag2 = make_float2(f.z, f.w);
+            } else {
+                ir = sc.ir[row];
+            }
+            uint32_t u[PANEL];
 #pragma unroll
-        for (int j = 0; j < PANEL; j += 2) {
-            const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), ir, mag2);
-            u[j] = __float_as_uint(f.x);
-            u[j + 1] = __float_as_uint(f.y);
-        }
-        if (any_tiny) {
-            // subnormal row factor: 1/r overflows; scale P and r by 2^64 (exact: |P| <= qmax r)
-            const float r = r_io[row];
-            if (r > 0.0f && r < FLT_MIN) {
-                const float irs = rcp_refined(r * 0x1p64f);
+            for (int j = 0; j < PANEL; j += 2) {
+                const float2 f = ffma2(make_float2(T[m][j], T[m][j + 1]), ir, mag2);
+                u[j] = __float_as_uint(f.x);
+                u[j + 1] = __float_as_uint(f.y);
+            }
+            if constexpr (decltype(tiny_rows)::value) {
+                // subnormal row factor: 1/r overflows; scale P and r by 2^64 (exact: |P| <= qmax r)
+                const float r = r_io[row];
+                if (r > 0.0f && r < FLT_MIN) {
+                    const float irs = rcp_refined(r * 0x1p64f);
 #pragma unroll
-                for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(fmaf(T[m][j] * 0x1p64f, irs, mag2.x));
+                    for (int j = 0; j < PANEL; ++j) u[j] = __float_as_uint(fmaf(T[m][j] * 0x1p64f, irs, mag2.x));
+                }
+            }
+            if constexpr (BITS == 0) {
+                uint8_t *seg = codes + panel * pb + row_seg_off(row, n8, n4);
+                const int wdt = row_width(row, n8, n4);
+                if (wdt == 8)
+                    pack_seg<8>(u, seg);
+                else if (wdt == 4)
+                    pack_seg<4>(u, seg);
+                else
+                    pack_seg<6>(u, seg);
+            } else {
+                pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
             }
         }
-        if constexpr (BITS == 0) {
-            uint8_t *seg = codes + panel * pb + row_seg_off(row, n8, n4);
-            const int wdt = row_width(row, n8, n4);
-            if (wdt == 8)
-                pack_seg<8>(u, seg);
-            else if (wdt == 4)
-                pack_seg<4>(u, seg);
-            else
-                pack_seg<6>(u, seg);
-        } else {
-            pack_seg<BITS>(u, codes + panel * panel_bytes(BITS) + row * seg_bytes(BITS));
-        }
-    }
+    };
+    if (any_tiny)
+        quantize_pack(std::true_type{});
+    else
+        quantize_pack(std::false_type{});
     // each warp stores its panel of codes and its slice of c (warp 0 also r)
     fence_proxy_async_smem();
     __syncwarp();
@@ -393,7 +411,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
 // (c0_j when a sum is not positive); codes = nearest levels of S / (r c), clipped.  With
 // P_ij = S_ij / r_i the sums are sum (w r^2) Q0 P and sum (w r^2) Q0^2, reduced over the warp
 // like the column dot products.
-template <int GATE, typename TIn, int BITS>
+template <int GATE, typename TIn, int BITS, bool ROWS>
 __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *stages, int i, bool has_next,
                                              const DecodeArgs &a, Scratch &sc, const TileIdx<4> &ix, int tid, int h,
                                              float cprime, TIn alpha_next_raw, bool ok, float *r_io, float *c_io,
@@ -444,7 +462,7 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
         sc.fit[tid] = make_float4(ir, ir, wr2, wr2);
         fence_proxy_async_smem();                  // r is bulk-stored from the stage by warp 0
     } else if (has_next && sc.meta[(i + 1) % kStages].valid) {
-        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, sc.meta[(i + 1) % kStages].bits,
+        row_table<GATE, TIn, ROWS>(stages + ((i + 1) % kStages) * stage_bytes_of<GATE>(), a, sc.meta[(i + 1) % kStages].bits,
                              sc.meta[(i + 1) % kStages].head, to_f32(alpha_next_raw), sc, tid);
     }
     __syncthreads();
@@ -533,7 +551,7 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
 
 // Per-CTA state of the item loop.  The loop runs in three pieces, one per bit width
 // (the heads are visited grouped by width), so each piece is compiled for one width.
-template <int GATE, typename TIn, bool IMPACT>
+template <int GATE, typename TIn, bool IMPACT, bool ROWS>
 struct ItemLoop {
     const DecodeArgs &a;
     Scratch &sc;
@@ -563,7 +581,7 @@ struct ItemLoop {
         sc.prod_b = pc.b;
         sc.prod_h = pc.h;
         if (j + 1 < count) slot_next = __ldg(a.slot_ids + pc.b);
-        uint8_t *stage = stages + st * a.stage_bytes;
+        uint8_t *stage = stages + st * stage_bytes_of<GATE>();
         StageMeta &mt = sc.meta[st];
         if (slot < 0 || slot >= a.num_slots) {
             mt.valid = 0;
@@ -581,11 +599,11 @@ struct ItemLoop {
             const uint32_t io = DK * esz;
             mbar_arrive_expect_tx(&sc.full[st], bb + 3 * io + (GATE == STEPQ_GATE_KDA ? io : 0u));
             bulk_g2s(stage, a.pool + mt.dst, bb, &sc.full[st]);
-            bulk_g2s(stage + a.blk_cap, static_cast<const uint8_t *>(a.q) + kqrow * io, io, &sc.full[st]);
-            bulk_g2s(stage + a.blk_cap + kIoBytes, static_cast<const uint8_t *>(a.k) + kqrow * io, io, &sc.full[st]);
-            bulk_g2s(stage + a.blk_cap + 2 * kIoBytes, static_cast<const uint8_t *>(a.v) + bh * io, io, &sc.full[st]);
+            bulk_g2s(stage + kBlkCap, static_cast<const uint8_t *>(a.q) + kqrow * io, io, &sc.full[st]);
+            bulk_g2s(stage + kBlkCap + kIoBytes, static_cast<const uint8_t *>(a.k) + kqrow * io, io, &sc.full[st]);
+            bulk_g2s(stage + kBlkCap + 2 * kIoBytes, static_cast<const uint8_t *>(a.v) + bh * io, io, &sc.full[st]);
             if (GATE == STEPQ_GATE_KDA)
-                bulk_g2s(stage + a.blk_cap + 3 * kIoBytes, static_cast<const uint8_t *>(a.alpha) + bh * io, io,
+                bulk_g2s(stage + kBlkCap + 3 * kIoBytes, static_cast<const uint8_t *>(a.alpha) + bh * io, io,
                          &sc.full[st]);
         }
     }
@@ -628,12 +646,12 @@ struct ItemLoop {
                 if (alive) {
                     const StageMeta mn = sc.meta[(i + 1) % kStages];
                     if (has_next && mn.valid && tid >= DK)
-                        row_table<GATE, TIn>(stages + ((i + 1) % kStages) * a.stage_bytes, a, mn.bits, mn.head,
+                        row_table<GATE, TIn, ROWS>(stages + ((i + 1) % kStages) * stage_bytes_of<GATE>(), a, mn.bits, mn.head,
                                              to_f32(alpha_raw), sc, tid);
                     __syncthreads();
                 }
             } else {
-                alive = decode_item<GATE, TIn, BITS, IMPACT>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
+                alive = decode_item<GATE, TIn, BITS, IMPACT, ROWS>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
                                                      alpha_raw, ok);
             }
             if (!alive) return false;
@@ -651,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *stages = smem;
-    Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * a.stage_bytes);
+    Scratch &sc = *reinterpret_cast<Scratch *>(smem + kStages * stage_bytes_of<GATE>());
 
     const int tid = threadIdx.x;
     const long long total = (long long)a.n * a.Hq;
@@ -682,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     }
     __syncthreads();
 
-    ItemLoop<GATE, TIn, IMPACT> L(a, sc, stages, tid, count);
+    ItemLoop<GATE, TIn, IMPACT, ROWS> L(a, sc, stages, tid, count);
     L.cur = {int(first % a.n), int(first / a.n)};
     if (tid == 0) {
         sc.prod_b = L.cur.b;
@@ -701,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     {
         const StageMeta m0 = sc.meta[0];
         const float al0 = (GATE == STEPQ_GATE_GDN) ? to_f32(alpha_g[L.bh_cur]) : 1.0f;
-        if (m0.valid && tid >= DK) row_table<GATE, TIn>(stages, a, m0.bits, m0.head, al0, sc, tid);
+        if (m0.valid && tid >= DK) row_table<GATE, TIn, ROWS>(stages, a, m0.bits, m0.head, al0, sc, tid);
     }
     __syncthreads();
 
@@ -912,9 +930,8 @@ cudaError_t decode_configure(stepq_pool *p)
 {
     cudaError_t e = upload_tables();
     if (e != cudaSuccess) return e;
-    p->blk_cap = p->max_block;
-    const int io = (p->gate_mode == STEPQ_GATE_KDA ? 4 : 3) * kIoBytes;
-    p->stage_bytes = (p->blk_cap + io + 127) / 128 * 128;
+    p->blk_cap = kBlkCap;
+    p->stage_bytes = p->gate_mode == STEPQ_GATE_KDA ? stage_bytes_of<STEPQ_GATE_KDA>() : stage_bytes_of<STEPQ_GATE_GDN>();
     p->decode_smem = decode_smem_bytes(p->stage_bytes);
     if (p->gate_mode == STEPQ_GATE_GDN)
         return p->in_dtype == STEPQ_DTYPE_BF16 ? configure_one<STEPQ_GATE_GDN, uint16_t>(p)
@@ -942,8 +959,6 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
     a.y = y;
     a.flag = p->d_flag;
-    a.blk_cap = p->blk_cap;
-    a.stage_bytes = p->stage_bytes;
     a.Hq = p->H - p->npiv;
     a.impact = p->d_impact;
     a.head_blk = p->d_blk;
@@ -1112,12 +1127,11 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     int32_t *order = reinterpret_cast<int32_t *>(image + kNoallocOrderOffset);
     uint8_t *bits = image + kNoallocBitsOffset;
     long long stride = 0;
-    int max_block = 0, nord = 0;
+    int nord = 0;
     for (int h = 0; h < H; ++h) {
         off[h] = stride;
         bits[h] = desc->head_bits[h];
         stride += block_bytes(bits[h]);
-        if (block_bytes(bits[h]) > max_block) max_block = block_bytes(bits[h]);
     }
     for (int w = 4; w <= 8; w += 2)
         for (int h = 0; h < H; ++h)
@@ -1146,9 +1160,8 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta;
     a.y = y;
     a.flag = reinterpret_cast<int *>(nd->scratch + kNoallocFlagOffset);
-    a.blk_cap = max_block;
-    a.stage_bytes = (max_block + (desc->gate_mode == STEPQ_GATE_KDA ? 4 : 3) * kIoBytes + 127) / 128 * 128;
-    const size_t smem = decode_smem_bytes(a.stage_bytes);
+    const size_t smem = decode_smem_bytes(desc->gate_mode == STEPQ_GATE_KDA ? stage_bytes_of<STEPQ_GATE_KDA>()
+                                                                        : stage_bytes_of<STEPQ_GATE_GDN>());
     if (desc->gate_mode == STEPQ_GATE_GDN)
         e = desc->in_dtype == STEPQ_DTYPE_BF16 ? noalloc_launch<STEPQ_GATE_GDN, uint16_t>(a, nd->num_sms, smem, stream)
                                                : noalloc_launch<STEPQ_GATE_GDN, float>(a, nd->num_sms, smem, stream);
