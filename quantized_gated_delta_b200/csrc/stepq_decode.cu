@@ -152,6 +152,18 @@ __device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs
     if ((t & 31) == 0) sc.kqw[(t >> 5) - 4] = kq;
 }
 
+// Lane 0 of each warp, after issuing its stores of item i: close them as one bulk group, then
+// wait until the warp's stores of item i-1 have read their stage and release that stage to
+// the producer (one arrival per warp on its empty barrier).
+__device__ __forceinline__ void retire_stores(Scratch &sc, int i)
+{
+    bulk_commit();
+    if (i >= 1) {
+        bulk_wait_read<1>();
+        mbar_arrive(&sc.empty[(i - 1) % kStages]);
+    }
+}
+
 // One state: the register tile through the row-maxima exchange, the row finalization /
 // next row table, then quantization, packing and the per-warp stores.  Returns false on
 // every thread when some thread saw a failed wait.
@@ -401,6 +413,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         bulk_s2g(dst + panel * pb, codes + panel * pb, uint32_t(pb));
         bulk_s2g(dst + cbytes + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
         if (panel == 0) bulk_s2g(dst + cbytes, r_io, 4 * DK);
+        retire_stores(sc, i);
     }
     return true;
 }
@@ -545,6 +558,7 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
         bulk_s2g(dst + panel * panel_bytes(BITS), codes + panel * panel_bytes(BITS), panel_bytes(BITS));
         bulk_s2g(dst + codes_bytes(BITS) + 4 * DK + 4 * PANEL * panel, c_io + PANEL * panel, 4 * PANEL);
         if (panel == 0) bulk_s2g(dst + codes_bytes(BITS), r_io, 4 * DK);
+        retire_stores(sc, i);
     }
     return true;
 }
@@ -617,10 +631,6 @@ struct ItemLoop {
         const TIn *beta_g = static_cast<const TIn *>(a.beta);
         for (; i < i_end; ++i) {
             const int st = i % kStages;
-            if (lane == 0 && i >= 2) {
-                bulk_wait_read<1>();                  // this warp's stores of item i-2 have read their stage
-                mbar_arrive(&sc.empty[(i - 2) % kStages]);
-            }
             if (tid == 0 && i + 2 < count) {
                 if (i + 2 >= kStages)                // stage (i+2)%4 last held item i-2
                     ok &= mbar_wait_bounded(&sc.empty[(i + 2) % kStages], uint32_t((i - 2) / kStages) & 1u);
@@ -649,13 +659,13 @@ struct ItemLoop {
                         row_table<GATE, TIn, ROWS>(stages + ((i + 1) % kStages) * stage_bytes_of<GATE>(), a, mn.bits, mn.head,
                                              to_f32(alpha_raw), sc, tid);
                     __syncthreads();
+                    if (lane == 0) retire_stores(sc, i);     // an empty group keeps one group per item
                 }
             } else {
                 alive = decode_item<GATE, TIn, BITS, IMPACT, ROWS>(stages, i, has_next, a, sc, ix, tid, bh_cur, beta_cur, kq,
                                                      alpha_raw, ok);
             }
             if (!alive) return false;
-            if (lane == 0) bulk_commit();
             cur = nxt;
             bh_cur = bh_next;
             beta_cur = to_f32(beta_raw);
