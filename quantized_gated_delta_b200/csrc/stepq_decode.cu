@@ -175,7 +175,7 @@ __device__ __forceinline__ bool refit_impact(float (&T)[kRows][PANEL], uint8_t *
 
 template <int GATE, typename TIn, int BITS, bool IMPACT, bool ROWS>
 __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_next, const DecodeArgs &a, Scratch &sc,
-                                            const TileIdx<4> &ix, int tid, long long bh, float beta, float kq,
+                                            const TileIdx<4> &ix, int tid, int bh, float beta, float kq,
                                             TIn alpha_next_raw, bool ok)
 {
     uint8_t *stage = stages + (i % kStages) * stage_bytes_of<GATE>();
@@ -187,7 +187,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     const int panel = ix.panel;
     const bool upper = (lane & 16) != 0;            // lanes holding the q-weighted sums first
     const int col = lane & 15;                      // the column this lane finalizes
-    const int head = int(bh % a.H);
+    const int head = sc.meta[i % kStages].head;
     int n8 = 0, n4 = 0, pb = panel_bytes(BITS ? BITS : 4);
     if constexpr (BITS == 0) {
         n8 = a.row_n8[head];
@@ -261,7 +261,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     const float val = cprime * A[0];
     const float delta = beta * (to_f32(vs[panel * PANEL + col]) - val);
     const float dpair = __shfl_xor_sync(kFull, delta, 16);
-    st_global_if(upper, a.y + bh * DV + panel * PANEL + col, fmaf(dpair, kq, val));
+    st_global_if(upper, a.y + (long long)bh * DV + panel * PANEL + col, fmaf(dpair, kq, val));
     st_shared_if(!upper, sc.xd + panel * PANEL + col, div_refined(delta, cprime));
     __syncwarp();
     float dd[PANEL];
@@ -284,7 +284,7 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
         }
     }
     if constexpr (IMPACT && BITS != 0)          // heads with per-row widths keep the clip-free fit
-        return refit_impact<GATE, TIn, BITS, ROWS>(T, stages, i, has_next, a, sc, ix, tid, int(bh % a.H), cprime,
+        return refit_impact<GATE, TIn, BITS, ROWS>(T, stages, i, has_next, a, sc, ix, tid, head, cprime,
                                              alpha_next_raw, ok, r_io, c_io, codes);
     // column maxima: over the thread's rows, then a warp-wide max per column; the 16
     // results go through shared memory (the d' buffer, already read) to the column lanes
@@ -573,7 +573,7 @@ struct ItemLoop {
     TileIdx<4> ix;
     int tid, lane, count;
     Cursor cur;
-    long long bh_cur;
+    int bh_cur;                         // b * H + h of the current item
     float beta_cur;
     bool ok;
     int slot_next;                      // producer: prefetched slot id of the next item to issue
@@ -640,7 +640,7 @@ struct ItemLoop {
             Cursor nxt = cur;
             nxt.advance(a);
             const bool has_next = i + 1 < count;
-            const long long bh_next = has_next ? (long long)nxt.b * a.H + sc.hord[nxt.h] : 0;
+            const int bh_next = has_next ? nxt.b * a.H + sc.hord[nxt.h] : 0;
             TIn beta_raw = TIn(0), alpha_raw = TIn(0);            // converted when used
             if (has_next) {
                 beta_raw = beta_g[bh_next];
@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
     // ---- prologue: the first state's row table
     const TIn *alpha_g = static_cast<const TIn *>(a.alpha);
     const TIn *beta_g = static_cast<const TIn *>(a.beta);
-    L.bh_cur = (long long)L.cur.b * a.H + sc.hord[L.cur.h];
+    L.bh_cur = L.cur.b * a.H + sc.hord[L.cur.h];
     L.beta_cur = to_f32(beta_g[L.bh_cur]);
     L.ok = mbar_wait_bounded(&sc.full[0], 0u);
     {

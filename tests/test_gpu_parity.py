@@ -329,25 +329,30 @@ def test_zero_requests_and_invalid_arguments(S):
     assert gp.get_error() == 0
 
 
-def test_host_buffer_steps_match_device_steps(S):
+@pytest.mark.parametrize("gate,dtype", [(0, 1), (1, 0)], ids=["gdn-bf16", "kda-fp32"])
+def test_host_buffer_steps_match_device_steps(S, gate, dtype):
     """stepq_decode_step_host (slot ids, inputs and y in host memory; copy-in, step and
     copy-out of consecutive calls overlapped through two staging buffers) gives outputs and
     states bit-identical to stepq_decode_step on device buffers, call after call: six calls
     enqueued back to back on pinned buffers, then one on pageable buffers, then a larger
-    batch that regrows the staging buffers."""
+    batch that regrows the staging buffers.  GDN with bf16 inputs and KDA (per-channel gate
+    vectors in the staging buffer) with fp32 inputs."""
     rng = np.random.default_rng(5)
     bits, H, Hk, num_slots = [4, 6, 8, 6], 4, 2, 12
     ids_all = np.array([6, 1, 3, 0, 5, 9, 11, 2], np.int32)
     S0 = torch.from_numpy(random_states(rng, len(ids_all), H)).cuda()
-    pools = [S.Pool(num_slots, bits, Hk, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_BF16) for _ in range(2)]
+    pools = [S.Pool(num_slots, bits, Hk, gate, dtype) for _ in range(2)]
     for gp in pools:
         gp.load_fp32(slots_t(ids_all), S0)
 
     def inputs(n):
+        ashape = (n, H, 128) if gate == S.STEPQ_GATE_KDA else (n, H)
         x = dict(q=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
                  k=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
                  v=rng.standard_normal((n, H, 128)).astype(f32),
-                 alpha=rng.uniform(0.8, 1, (n, H)).astype(f32), beta=rng.uniform(0, 1, (n, H)).astype(f32))
+                 alpha=rng.uniform(0.8, 1, ashape).astype(f32), beta=rng.uniform(0, 1, (n, H)).astype(f32))
+        if dtype == S.STEPQ_DTYPE_F32:
+            return {key: torch.from_numpy(val) for key, val in x.items()}
         return {key: torch.from_numpy(W.to_bf16_bits(val).view(np.int16)) for key, val in x.items()}
 
     plan = [(5, True)] * 6 + [(5, False), (8, True)]
