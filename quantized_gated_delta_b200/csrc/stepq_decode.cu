@@ -105,6 +105,7 @@ struct Scratch {
     long long hoff[kMaxHeads];      // head block offsets inside a slot
     int32_t hord[kMaxHeads];        // head processing order
     uint8_t hbits[kMaxHeads];       // head widths
+    uint8_t hkey[kMaxHeads];        // key head of each value head (h / group)
     StageMeta meta[kStages];
     int prod_b, prod_h;             // producer cursor
     uint64_t full[kStages];
@@ -590,7 +591,7 @@ struct ItemLoop {
         const int st = j % kStages;
         const int slot = slot_next;
         Cursor pc = {sc.prod_b, sc.prod_h};
-        const int b = pc.b, h = sc.hord[pc.h], g = h / a.group;
+        const int b = pc.b, h = sc.hord[pc.h], g = sc.hkey[h];
         pc.advance(a);
         sc.prod_b = pc.b;
         sc.prod_h = pc.h;
@@ -707,6 +708,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
         sc.hoff[h] = a.head_off[h];
         sc.hord[h] = a.head_order[h];
         sc.hbits[h] = a.head_bits[h];
+        sc.hkey[h] = uint8_t(h / a.group);
     }
     __syncthreads();
 
