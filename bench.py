@@ -212,6 +212,25 @@ def _cpu_model() -> str:
     return "unknown"
 
 
+def slot_stride_of(bits) -> int:
+    """Bytes of one slot: per head, codes + r + c (an FP16 pivot head: 2 bytes per value)."""
+    return sum(2 * 128 * 128 if int(b) == 16 else 128 * 128 * int(b) // 8 + 8 * 128 for b in bits)
+
+
+def pool_config(w, bits, row_bits, fit, world, slot_stride, nsets):
+    """The `config` of a bench line on the single-pool workloads (both arms)."""
+    return {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s%s"
+                        % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
+                           "".join(str(int(b)) for b in bits) if row_bits is None else "per key row (4/6/8: %s)"
+                           % "/".join(str(int(np.sum(row_bits == x))) for x in (4, 6, 8)),
+                           ", impact-weighted fit" if fit == "impact" else ""),
+            "avg_bits": float(np.mean(bits if row_bits is None else row_bits)),
+            "parallelism": "dp%d (independent pools)" % world,
+            "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
+                  % (w.B * slot_stride / 1e6),
+            "input_sets": nsets}
+
+
 def run_reference(args):
     """Reference arm: the oracle, as it stands, timed on the host cores.  Each step is a
     bounded sample of the workload's requests, sized so the whole run takes a few minutes."""
@@ -245,7 +264,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name},
+            "data": "synthetic",
+            "config": pool_config(w, bits, None, "clipfree", args.gpus, slot_stride_of(bits), args.input_sets),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "%d requests x %d heads per step, %d steps of %s"
                                        % (len(sl), w.H, args.steps, w.name)},
@@ -499,16 +519,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s%s"
-                       % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
-                          "".join(str(int(b)) for b in bits) if row_bits is None else "per key row (4/6/8: %s)"
-                          % "/".join(str(int(np.sum(row_bits == x))) for x in (4, 6, 8)),
-                          ", impact-weighted fit" if args.fit == "impact" else ""),
-                       "avg_bits": float(np.mean(bits if row_bits is None else row_bits)),
-                       "parallelism": "dp%d (independent pools)" % world,
-                       "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
-                             % (w.B * pool.slot_stride / 1e6),
-                       "input_sets": nsets},
+            "config": pool_config(w, bits, row_bits, args.fit, world, pool.slot_stride, nsets),
             "achieved_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,
