@@ -100,6 +100,39 @@ def fp16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(key(a) - key(b))
 
 
+TIE_DIST = 2e-4        # code units: a few fp32 ulps of S / (r c) at qmax, plus the r / c ulps allowed
+
+
+def flips_off_tie(gpu_bytes, ora_before, bits, Hk, x, dk=128, dv=128):
+    """Codes of a GPU step that differ from the oracle's and are not at a rounding tie.
+
+    For each state and head the oracle's own step (from the slot bytes before the step,
+    ora_before [n, slot_stride], and the inputs x of those n requests, GDN) gives the
+    updated state before rounding and the fitted r, c; a code may differ by one only where
+    |S / (r c)| lies within TIE_DIST of a half-integer (both roundings are then correct).
+    Returns (count of differing codes off a tie, largest code difference)."""
+    offs, _ = O.head_offsets(bits, dk, dv)
+    H = len(bits)
+    off_tie, worst = 0, 0
+    for s in range(gpu_bytes.shape[0]):
+        for h, b in enumerate(bits):
+            b = int(b)
+            n = O.block_bytes(b, dk, dv)
+            Q0, r0, c0 = O.split_block(ora_before[s, offs[h]:offs[h] + n], b, dk, dv)
+            g = h // (H // Hk)
+            out = O.step_state(Q0, r0, c0, b, x["q"][s, g], x["k"][s, g], x["v"][s, h], x["alpha"][s, h],
+                               float(x["beta"][s, h]))
+            Qg = O.split_block(gpu_bytes[s, offs[h]:offs[h] + n], b, dk, dv)[0]
+            d = np.abs(Qg.astype(np.int64) - out["Q"])
+            worst = max(worst, int(d.max()))
+            den = np.outer(out["r"].astype(np.float64), out["c"].astype(np.float64))
+            S32 = out["S_pre"].astype(np.float32).astype(np.float64)
+            t = np.abs(np.divide(S32, den, out=np.zeros_like(S32), where=den > 0))
+            at_tie = np.abs(t - np.floor(t) - 0.5) < TIE_DIST
+            off_tie += int(np.sum((d > 0) & ~at_tie))
+    return off_tie, worst
+
+
 def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv=128, row_bits=None) -> dict:
     """Compare slot images [n, slot_stride] head by head (FP16 pivot heads by binary16 ulps;
     heads of width 0 by their per-key-row widths row_bits [H, dk])."""

@@ -240,6 +240,73 @@ def test_pivot_heads_load_dump_and_step(S):
         assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
 
 
+def _unit_rows(rng, shape):
+    x = rng.standard_normal(shape + (128,))
+    return (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(f32)
+
+
+def test_max_heads_vs_oracle(S):
+    """The largest pool shape a call accepts in heads: H = 256 value heads (every width, FP16
+    pivot heads among them) on 128 key heads; one step from random states, every state
+    against the oracle."""
+    rng = np.random.default_rng(21)
+    H, Hk, n = 256, 128, 3
+    bits = [(4, 6, 8, 16, 6, 4, 8, 6)[h % 8] for h in range(H)]
+    st = random_states(rng, n, H, steps=4)
+    ids = np.array([4, 0, 2], np.int32)
+    op = O.OraclePool(5, bits, Hk)
+    op.load_fp32(ids, st)
+    x = dict(q=_unit_rows(rng, (n, Hk)), k=_unit_rows(rng, (n, Hk)),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.7, 1, (n, H)).astype(f32), beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+    yg, sg, err = _run_gpu(S, bits, Hk, 0, S.STEPQ_DTYPE_F32, x, op.slot_bytes(ids), ids, 5)
+    assert err == 0
+    yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    res = PH.compare_slots(sg, op.slot_bytes(ids), bits)
+    assert PH.pivots_ok(res), res
+    assert res["max_code_diff"] <= 1 and res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
+    assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
+    assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
+
+
+def test_max_requests_sampled_vs_oracle(S):
+    """The largest request count a call accepts: n = 65535 requests on a 65535-slot pool
+    (every slot, in a random order), one launch; the oracle follows the first and the last
+    request, four in between (loaded with random states) and two that start from the zeroed
+    pool.  A state stepped from zero is rank one, so every row of a column carries the same
+    code and a column at a rounding tie puts 128 elements at that tie at once: the codes are
+    checked element by element instead of by a flip rate -- each code equals the oracle's,
+    or differs by one where the oracle's S / (r c) is at a tie."""
+    rng = np.random.default_rng(22)
+    n, H, Hk, bits = 65535, 2, 1, [4, 8]
+    slot_ids = rng.permutation(n).astype(np.int32)
+    loaded = np.array([0, 1, 20000, 40000, 65533, 65534])
+    fresh = np.array([7, 50001])
+    sample = np.concatenate([loaded, fresh])
+    st = random_states(rng, len(loaded), H, steps=8)
+    op = O.OraclePool(len(sample), bits, Hk)
+    op.load_fp32(np.arange(len(loaded), dtype=np.int32), st)
+    gp = S.Pool(n, bits, Hk, S.STEPQ_GATE_GDN, S.STEPQ_DTYPE_BF16)
+    load_bytes(gp, slot_ids[loaded], op.slot_bytes(np.arange(len(loaded))))
+    x = dict(q=_unit_rows(rng, (n, Hk)), k=_unit_rows(rng, (n, Hk)),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.7, 1, (n, H)).astype(f32), beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+    x = {key: W.round_bf16(val) for key, val in x.items()}
+    tx = {key: dev(W.to_bf16_bits(val).view(np.int16)) for key, val in x.items()}
+    y = torch.empty((n, H, 128), device="cuda")
+    gp.decode_step(slots_t(slot_ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    assert gp.get_error() == 0
+    before = op.slot_bytes(np.arange(len(sample)))
+    xs = {key: x[key][sample] for key in ("q", "k", "v", "alpha", "beta")}
+    yo = op.decode_step(np.arange(len(sample), dtype=np.int32), xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"])
+    sg = dump_bytes(gp, slot_ids[sample])
+    res = PH.compare_slots(sg, op.slot_bytes(np.arange(len(sample))), bits)
+    assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
+    off_tie, worst = PH.flips_off_tie(sg, before, bits, Hk, xs)
+    assert worst <= 1 and off_tie == 0
+    assert PH.y_max_rel(y[torch.from_numpy(sample).cuda()].cpu().numpy(), yo) <= PH.Y_MAX_REL
+
+
 def _run_gpu(S, bits, Hk, gate, dtype, x, init_bytes, ids, num_slots):
     gp = S.Pool(num_slots, bits, Hk, gate, dtype)
     load_bytes(gp, ids, init_bytes)
