@@ -14,6 +14,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -69,12 +70,22 @@ def peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+def _code_only(src: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed (string literals in
+    these files hold no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def kernel_source_hash(csrc: str | None = None) -> str:
+    """Hash of the library's code (comments and layout excluded): a recorded ncu traffic
+    figure is reported only for the code it was measured on."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "quantized_gated_delta_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "quantized_gated_delta_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
