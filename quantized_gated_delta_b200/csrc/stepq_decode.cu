@@ -711,6 +711,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
         sc.hkey[h] = uint8_t(h / a.group);
     }
     __syncthreads();
+    // everything above reads only the pool's tables; the states, the inputs and y may still be
+    // in use by the previous grid of the stream when this one was launched as its dependent
+    grid_dependency_wait();
+    // the next grid may launch now: its CTAs become resident only as this grid's CTAs exit
+    if (tid == 0) grid_launch_dependents();
 
     ItemLoop<GATE, TIn, IMPACT, ROWS> L(a, sc, stages, tid, count);
     L.cur = {int(first % a.n), int(first / a.n)};
@@ -910,20 +915,33 @@ cudaError_t upload_tables()
     return cudaMemcpyToSymbol(kInvPos, h, sizeof(h));
 }
 
-template <int GATE, typename TIn>
-void launch_variant(bool impact, bool rows, int grid, size_t smem, cudaStream_t stream, const DecodeArgs &a)
+// The decode kernel is launched as a programmatic dependent of the previous kernel in the
+// stream: its CTAs may start (shared-memory setup, head tables) while that kernel's last
+// CTAs finish, and wait for it before touching states, inputs or y.
+template <int GATE, typename TIn, bool IMPACT, bool ROWS>
+cudaError_t launch_dependent(int grid, size_t smem, cudaStream_t stream, const DecodeArgs &a)
 {
-    if (impact) {
-        if (rows)
-            decode_kernel<GATE, TIn, true, true><<<grid, kThreads, smem, stream>>>(a);
-        else
-            decode_kernel<GATE, TIn, true, false><<<grid, kThreads, smem, stream>>>(a);
-    } else {
-        if (rows)
-            decode_kernel<GATE, TIn, false, true><<<grid, kThreads, smem, stream>>>(a);
-        else
-            decode_kernel<GATE, TIn, false, false><<<grid, kThreads, smem, stream>>>(a);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<GATE, TIn, IMPACT, ROWS>, a);
+}
+
+template <int GATE, typename TIn>
+cudaError_t launch_variant(bool impact, bool rows, int grid, size_t smem, cudaStream_t stream, const DecodeArgs &a)
+{
+    if (impact)
+        return rows ? launch_dependent<GATE, TIn, true, true>(grid, smem, stream, a)
+                    : launch_dependent<GATE, TIn, true, false>(grid, smem, stream, a);
+    return rows ? launch_dependent<GATE, TIn, false, true>(grid, smem, stream, a)
+                : launch_dependent<GATE, TIn, false, false>(grid, smem, stream, a);
 }
 
 void count_widths(const uint8_t *bits, int H, DecodeArgs &a)
@@ -987,18 +1005,14 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
         a.step_h = grid / n;
         const size_t sm = p->decode_smem;
         const bool rows = p->d_perm != nullptr;
-        if (p->gate_mode == STEPQ_GATE_GDN) {
-            if (p->in_dtype == STEPQ_DTYPE_BF16)
-                launch_variant<STEPQ_GATE_GDN, uint16_t>(a.impact != nullptr, rows, grid, sm, stream, a);
-            else
-                launch_variant<STEPQ_GATE_GDN, float>(a.impact != nullptr, rows, grid, sm, stream, a);
-        } else {
-            if (p->in_dtype == STEPQ_DTYPE_BF16)
-                launch_variant<STEPQ_GATE_KDA, uint16_t>(a.impact != nullptr, rows, grid, sm, stream, a);
-            else
-                launch_variant<STEPQ_GATE_KDA, float>(a.impact != nullptr, rows, grid, sm, stream, a);
-        }
-        const cudaError_t e = cudaGetLastError();
+        const bool imp = a.impact != nullptr;
+        cudaError_t e;
+        if (p->gate_mode == STEPQ_GATE_GDN)
+            e = p->in_dtype == STEPQ_DTYPE_BF16 ? launch_variant<STEPQ_GATE_GDN, uint16_t>(imp, rows, grid, sm, stream, a)
+                                                : launch_variant<STEPQ_GATE_GDN, float>(imp, rows, grid, sm, stream, a);
+        else
+            e = p->in_dtype == STEPQ_DTYPE_BF16 ? launch_variant<STEPQ_GATE_KDA, uint16_t>(imp, rows, grid, sm, stream, a)
+                                                : launch_variant<STEPQ_GATE_KDA, float>(imp, rows, grid, sm, stream, a);
         if (e != cudaSuccess) return e;
     }
     if (p->npiv > 0) {
