@@ -106,6 +106,10 @@ struct Scratch {
     int32_t hord[kMaxHeads];        // head processing order
     uint8_t hbits[kMaxHeads];       // head widths
     uint8_t hkey[kMaxHeads];        // key head of each value head (h / group)
+    // heads with per-key-row widths (pools that have such heads): padded panel bytes and the
+    // counts of 8-bit and 4-bit rows
+    int32_t rpb[kMaxHeads];
+    uint8_t rn8[kMaxHeads], rn4[kMaxHeads];
     StageMeta meta[kStages];
     int prod_b, prod_h;             // producer cursor
     uint64_t full[kStages];
@@ -134,7 +138,7 @@ __device__ __forceinline__ void row_table(const uint8_t *stage, const DecodeArgs
 {
     const int i = t - 128;                          // stored row (the key row unless bits == 0)
     const bool rows = ROWS && bits == 0;            // heads with per-key-row widths exist only in ROWS pools
-    const float *r = reinterpret_cast<const float *>(stage + (rows ? 8 * a.row_pb[head] : codes_bytes(bits)));
+    const float *r = reinterpret_cast<const float *>(stage + (rows ? NPANEL * sc.rpb[head] : codes_bytes(bits)));
     const int key = rows ? int(a.row_perm[head * DK + i]) : i;
     const TIn *qs = reinterpret_cast<const TIn *>(stage + kBlkCap);
     const TIn *ks = reinterpret_cast<const TIn *>(stage + kBlkCap + kIoBytes);
@@ -191,9 +195,9 @@ __device__ __forceinline__ bool decode_item(uint8_t *stages, int i, bool has_nex
     const int head = sc.meta[i % kStages].head;
     int n8 = 0, n4 = 0, pb = panel_bytes(BITS ? BITS : 4);
     if constexpr (BITS == 0) {
-        n8 = a.row_n8[head];
-        n4 = a.row_n4[head];
-        pb = a.row_pb[head];
+        n8 = sc.rn8[head];
+        n4 = sc.rn4[head];
+        pb = sc.rpb[head];
     }
     const int cbytes = BITS ? codes_bytes(BITS) : 8 * pb;
 
@@ -604,7 +608,8 @@ struct ItemLoop {
             mbar_arrive(&sc.full[st]);
         } else {
             const int bits = sc.hbits[h];
-            const uint32_t bb = bits ? uint32_t(block_bytes(bits)) : uint32_t(a.head_blk[h]);
+            const uint32_t bb = (ROWS && bits == 0) ? uint32_t(NPANEL * sc.rpb[h] + 4 * DK + 4 * DV)
+                                                    : uint32_t(block_bytes(bits));
             const long long bh = (long long)b * a.H + h;
             const long long kqrow = (long long)b * a.Hk + g;
             mt.valid = 1;
@@ -709,6 +714,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a)
         sc.hord[h] = a.head_order[h];
         sc.hbits[h] = a.head_bits[h];
         sc.hkey[h] = uint8_t(h / a.group);
+        if constexpr (ROWS) {
+            sc.rpb[h] = a.row_pb[h];
+            sc.rn8[h] = a.row_n8[h];
+            sc.rn4[h] = a.row_n4[h];
+        }
     }
     __syncthreads();
     // everything above reads only the pool's tables; the states, the inputs and y may still be
