@@ -60,6 +60,9 @@ void free_pool(stepq_pool *p)
         if (p->ev_step[b]) cudaEventDestroy(p->ev_step[b]);
         if (p->ev_out[b]) cudaEventDestroy(p->ev_out[b]);
     }
+    if (p->ev_pfork) cudaEventDestroy(p->ev_pfork);
+    if (p->ev_pjoin) cudaEventDestroy(p->ev_pjoin);
+    if (p->s_piv) cudaStreamDestroy(p->s_piv);
     if (p->s_in) cudaStreamDestroy(p->s_in);
     if (p->s_out) cudaStreamDestroy(p->s_out);
     delete p;
@@ -225,6 +228,11 @@ int create_pool(const stepq_pool_desc *desc, const uint8_t *row_bits, stepq_pool
     if (e == cudaSuccess) e = cudaMalloc(&p->d_bits, size_t(p->H));
     if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * p->H);
     if (e == cudaSuccess) e = cudaMalloc(&p->d_flag, sizeof(int));
+    if (e == cudaSuccess && p->npiv > 0) {
+        e = cudaStreamCreateWithFlags(&p->s_piv, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_pfork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_pjoin, cudaEventDisableTiming);
+    }
     if (e == cudaSuccess) e = cudaMemset(p->d_pool, 0, size_t(p->total));
     if (e == cudaSuccess) e = cudaMemset(p->d_flag, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMemcpy(p->d_offs, p->offs.data(), sizeof(long long) * p->H, cudaMemcpyHostToDevice);

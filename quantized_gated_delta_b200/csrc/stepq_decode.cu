@@ -1008,6 +1008,14 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
     a.row_perm = p->d_perm;
     // items are dealt round-robin in head-major order, so the CTAs resident at any moment
     // work on one or two heads (one bit width: one code path in the instruction caches)
+    // FP16 pivot heads run on their own stream, forked here from the caller's stream: their
+    // kernel touches neither the quantized heads nor their rows of y, so it can take the SM
+    // slots that free up while the persistent decode grid finishes
+    const bool piv = p->npiv > 0;
+    if (piv) {
+        const cudaError_t e = cudaEventRecord(p->ev_pfork, stream);
+        if (e != cudaSuccess) return e;
+    }
     const long long total = (long long)n * a.Hq;
     if (total > 0) {
         const int grid = int(total < p->decode_grid ? total : p->decode_grid);
@@ -1025,19 +1033,27 @@ cudaError_t launch_decode(const stepq_pool *p, const int32_t *slot_ids, int n, c
                                                 : launch_variant<STEPQ_GATE_KDA, float>(imp, rows, grid, sm, stream, a);
         if (e != cudaSuccess) return e;
     }
-    if (p->npiv > 0) {
+    if (piv) {
+        cudaStream_t ps = p->s_piv;
+        cudaError_t e = cudaStreamWaitEvent(ps, p->ev_pfork, 0);
+        if (e != cudaSuccess) return e;
         const unsigned pgrid = unsigned(n) * unsigned(p->npiv);
         if (p->gate_mode == STEPQ_GATE_GDN) {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                pivot_kernel<STEPQ_GATE_GDN, uint16_t><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+                pivot_kernel<STEPQ_GATE_GDN, uint16_t><<<pgrid, kThreads, 0, ps>>>(a, p->npiv);
             else
-                pivot_kernel<STEPQ_GATE_GDN, float><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+                pivot_kernel<STEPQ_GATE_GDN, float><<<pgrid, kThreads, 0, ps>>>(a, p->npiv);
         } else {
             if (p->in_dtype == STEPQ_DTYPE_BF16)
-                pivot_kernel<STEPQ_GATE_KDA, uint16_t><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+                pivot_kernel<STEPQ_GATE_KDA, uint16_t><<<pgrid, kThreads, 0, ps>>>(a, p->npiv);
             else
-                pivot_kernel<STEPQ_GATE_KDA, float><<<pgrid, kThreads, 0, stream>>>(a, p->npiv);
+                pivot_kernel<STEPQ_GATE_KDA, float><<<pgrid, kThreads, 0, ps>>>(a, p->npiv);
         }
+        e = cudaGetLastError();
+        // join: everything after this step on the caller's stream sees the pivot heads done
+        if (e == cudaSuccess) e = cudaEventRecord(p->ev_pjoin, ps);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, p->ev_pjoin, 0);
+        return e;
     }
     return cudaGetLastError();
 }

@@ -35,6 +35,10 @@ struct stepq_pool {
     size_t decode_smem = 0;             // dynamic shared memory of the decode kernel
     int stage_bytes = 0;
     int blk_cap = 0;
+    // pools with FP16 pivot heads: the pivot kernel's stream, forked from and joined back to
+    // the caller's stream in every step (the two kernels share no data)
+    cudaStream_t s_piv = nullptr;
+    cudaEvent_t ev_pfork = nullptr, ev_pjoin = nullptr;
     // host-buffer decode (stepq_decode_step_host): two device staging buffers used in turn,
     // the copy-in and copy-out streams, and the events that chain copy-in -> step -> copy-out;
     // created on first use
