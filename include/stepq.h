@@ -151,7 +151,9 @@ STEPQ_API int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot
  *   alpha  [n, H] (GDN) or [n, H, d_k] (KDA): retention in (0, 1], not its logarithm
  *   beta   [n, H]
  *   y      [n, H, d_v] float32 output; rows of skipped (bad-slot) requests are not written
- * n = 0 is a valid no-op. */
+ * n = 0 is a valid no-op.  In a pool with FP16 pivot heads their kernel runs on a stream of
+ * the pool, forked from `stream` at the call and joined back to it: work enqueued on `stream`
+ * after the call sees every head updated.  The call may be captured in a CUDA graph. */
 STEPQ_API int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q,
                       const void *k, const void *v, const void *alpha, const void *beta, float *y,
                       stepq_stream stream);
