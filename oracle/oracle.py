@@ -503,7 +503,8 @@ def allocate_bits_dp_vec(half_life, distortion, cand, avg_bits):
         for ci in order:
             b = cand[ci]
             v = np.full(budget + 1, np.inf)
-            v[b:] = best[:budget + 1 - b] + w * _distortion(distortion, u, ci, cand)
+            if b <= budget:                      # a width above the whole budget never fits
+                v[b:] = best[:budget + 1 - b] + w * _distortion(distortion, u, ci, cand)
             better = v < nxt
             nxt = np.where(better, v, nxt)
             pick = np.where(better, ci, pick)

@@ -119,3 +119,16 @@ def test_pivot_allocator_equals_oracle(S):
         assert int(np.sum(got == 16)) == npv
     with pytest.raises(S.StepqError):
         S.stepq_allocate_bits_pivots([1.0, 2.0], None, (4, 6, 8), 6.0, 3)    # more pivots than units
+
+
+def test_vectorised_dp_equals_library_allocator_at_row_granularity(S):
+    """The per-key-row allocation of the KDA row-width workload (32 heads x 128 rows = 4096
+    units): the oracle's vectorised DP and the library's C++ allocator give the same widths."""
+    from quantized_gated_delta_b200 import workloads as W
+    w = W.make_workload(3, "rowbits")
+    hl = np.ravel(w.row_half_life[0])
+    assert hl.size == 4096
+    ref, _ = O.allocate_bits_dp_vec(list(hl), None, [4, 6, 8], 6.0)
+    got = S.stepq_allocate_bits(hl, None, (4, 6, 8), 6.0)
+    assert list(got) == ref
+    assert got.mean() == 6.0
