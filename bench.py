@@ -230,8 +230,9 @@ def slot_stride_of(bits) -> int:
     return sum(2 * 128 * 128 if int(b) == 16 else 128 * 128 * int(b) // 8 + 8 * 128 for b in bits)
 
 
-def pool_config(w, bits, row_bits, fit, world, slot_stride, nsets):
-    """The `config` of a bench line on the single-pool workloads (both arms)."""
+def pool_config(w, bits, row_bits, fit, world, slot_stride):
+    """The `config` of a bench line on the single-pool workloads (both arms: the workload only;
+    each arm reports the number of input batches it cycles in its own `input_sets` key)."""
     return {"workload": "%s: B=%d of %d slots, H=%d, Hk=%d, d_k=d_v=%d, %s inputs, bits %s%s"
                         % (w.name, w.B, w.num_slots, w.H, w.Hk, w.dk, w.dtype_name,
                            "".join(str(int(b)) for b in bits) if row_bits is None else "per key row (4/6/8: %s)"
@@ -240,8 +241,7 @@ def pool_config(w, bits, row_bits, fit, world, slot_stride, nsets):
             "avg_bits": float(np.mean(bits if row_bits is None else row_bits)),
             "parallelism": "dp%d (independent pools)" % world,
             "l2": "no flush: %.0f MB of packed state read and written per step (> 126 MB L2)"
-                  % (w.B * slot_stride / 1e6),
-            "input_sets": nsets}
+                  % (w.B * slot_stride / 1e6)}
 
 
 def run_reference(args):
@@ -278,7 +278,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": pool_config(w, bits, None, "clipfree", args.gpus, slot_stride_of(bits), args.input_sets),
+            "config": pool_config(w, bits, None, "clipfree", args.gpus, slot_stride_of(bits)),
+            "input_sets": len(xs),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "%d requests x %d heads per step, %d steps of %s"
                                        % (len(sl), w.H, args.steps, w.name)},
@@ -534,7 +535,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": pool_config(w, bits, row_bits, args.fit, world, pool.slot_stride, nsets),
+            "config": pool_config(w, bits, row_bits, args.fit, world, pool.slot_stride),
+            "input_sets": nsets,
             "achieved_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_source": peak_kind,

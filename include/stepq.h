@@ -20,9 +20,10 @@
  *   - Calls that take a stream enqueue work on it and return without synchronizing; an
  *     asynchronous CUDA fault surfaces as STEPQ_CUDA_ERROR on a later call.  A pool must
  *     not be used on two streams at once without synchronization by the caller.
- *   - slot_ids within one call must be distinct; duplicates give undefined results.  An
- *     out-of-range slot id is skipped by the kernels and raises the pool's sticky device
- *     flag (read with stepq_pool_get_error); kernels never trap.
+ *   - slot_ids within one call must be distinct; duplicates give undefined results (the
+ *     debug mode of stepq_pool_set_debug rejects them).  An out-of-range slot id is skipped by
+ *     the kernels and raises the pool's sticky device flag (read with stepq_pool_get_error);
+ *     kernels never trap.
  *
  * State and layout (shared by every call; the pages leave the format open)
  *   - value head h of request b lives in slot s = slot_ids[b]; key head g(h) = h / (H / H_k)
@@ -188,19 +189,23 @@ STEPQ_API int stepq_pool_host_wait(stepq_pool *pool, stepq_stream stream);
  * its own arena or caching allocator (and accounts for every byte), or code embedded where
  * new allocations are forbidden.  They keep the packed state themselves and pass it here;
  * no pool object exists.
- *   desc      as for stepq_pool_create (HOST, read during the call); num_heads <= 256, else
- *             STEPQ_UNSUPPORTED (the scratch holds the tables of at most 256 heads)
+ *   desc      as for stepq_pool_create (HOST, read during the call), with two limits that
+ *             give STEPQ_UNSUPPORTED: num_heads <= 256 (the scratch holds the tables of at
+ *             most 256 heads), and every head_bits[h] in {4, 6, 8} (FP16 pivot heads, width
+ *             16, are not taken: their kernel runs on a second stream of a pool)
  *   state     DEVICE, caller-owned, 128-byte aligned: num_slots slots in the pool layout
  *             (slot_stride = sum of the head block sizes), updated in place
  *   slot_ids, q, k, v, alpha, beta, y   as for stepq_decode_step
  *   flag_out  DEVICE, optional (may be NULL): receives this call's STEPQ_FLAG_* bits
- * The kernel's scratch (the flag word and the per-head tables, 3328 bytes) is a fixed device
+ * The kernel's scratch (the flag word and the per-head tables, 3584 bytes) is a fixed device
  * array inside the library, held by every GPU that loads it until the process exits.  Every
- * call rewrites it (flag cleared, tables refreshed) on `stream`; calls that overlap on the
- * GPU (other streams, other threads) share it and race.  The first call on each device
- * resolves the array's address and configures the kernel on that device, so it should come
- * before any stream capture.  The call allocates nothing (no cudaMalloc, cudaFree or
- * allocating library routine). */
+ * call rewrites it (flag cleared, tables refreshed) on `stream`, with a one-CTA kernel that
+ * receives the new contents as its launch argument, so the call reads no host memory
+ * asynchronously and does not wait on the host for earlier work of `stream`.  Calls that
+ * overlap on the GPU (other streams, other threads) share the array and race.  The first call
+ * on each device resolves the array's address and configures the kernels on that device,
+ * so it should come before any stream capture.  The call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine). */
 STEPQ_API int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *state, const int32_t *slot_ids,
                                         int32_t n, const void *q, const void *k, const void *v,
                                         const void *alpha, const void *beta, float *y, int32_t *flag_out,
@@ -226,6 +231,21 @@ STEPQ_API int stepq_pool_set_impact(stepq_pool *pool, const float *impact);
  * (HOST) receives the flag bits: STEPQ_FLAG_TIMEOUT when the path works.  The context stays
  * usable.  Synchronizes `stream`. */
 STEPQ_API int stepq_check_wait_timeout(int32_t *flag_out, stepq_stream stream);
+
+/* Debug checks of a pool, off by default.  With STEPQ_DEBUG_SLOTS, every call of the pool that
+ * takes slot_ids rejects duplicate or out-of-range ids with STEPQ_INVALID_ARG before any
+ * device work (without it, duplicates give undefined results and an out-of-range id is
+ * skipped by the kernels and flagged).  For device slot_ids the check copies them to the host
+ * and synchronizes the call's stream, so a pool in this mode is for development runs, not for
+ * stream capture; stepq_decode_step_host checks its host ids directly.  flags = 0 turns the
+ * checks off; unknown flag bits give STEPQ_INVALID_ARG.  The paper has no counterpart. */
+enum { STEPQ_DEBUG_SLOTS = 1 };
+STEPQ_API int stepq_pool_set_debug(stepq_pool *pool, int32_t flags);
+
+/* The same check on a HOST array: STEPQ_OK when slot_ids[0 .. n) are distinct and each lies in
+ * [0, num_slots), else STEPQ_INVALID_ARG (also for n < 0, num_slots <= 0, or a null array
+ * with n > 0). */
+STEPQ_API int stepq_check_slot_ids(const int32_t *slot_ids, int32_t n, int32_t num_slots);
 
 /* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
  * Synchronizes the device. */

@@ -40,6 +40,41 @@ int check_slots(const stepq_pool *p, const int32_t *slot_ids, int32_t n)
     return check_device(p);
 }
 
+// Distinct ids in [0, num_slots) (host array).
+int host_check_slot_ids(const int32_t *ids, int32_t n, int32_t num_slots)
+{
+    if (n < 0 || num_slots <= 0 || (n > 0 && !ids)) return STEPQ_INVALID_ARG;
+    std::vector<uint8_t> seen;
+    try {
+        seen.assign(size_t(num_slots), 0);
+    } catch (...) {
+        return STEPQ_OUT_OF_MEMORY;
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        const int32_t s = ids[i];
+        if (s < 0 || s >= num_slots || seen[size_t(s)]) return STEPQ_INVALID_ARG;
+        seen[size_t(s)] = 1;
+    }
+    return STEPQ_OK;
+}
+
+// Debug mode (STEPQ_DEBUG_SLOTS): copy a call's device slot ids to the host and check them
+// before any device work of the call (synchronizes `stream`).
+int debug_check_slots(const stepq_pool *p, const int32_t *slot_ids, int32_t n, cudaStream_t stream)
+{
+    if (!(p->debug & STEPQ_DEBUG_SLOTS) || n == 0) return STEPQ_OK;
+    std::vector<int32_t> h;
+    try {
+        h.resize(size_t(n));
+    } catch (...) {
+        return STEPQ_OUT_OF_MEMORY;
+    }
+    cudaError_t e = cudaMemcpyAsync(h.data(), slot_ids, sizeof(int32_t) * size_t(n), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return status_of(e);
+    return host_check_slot_ids(h.data(), n, p->num_slots);
+}
+
 void free_pool(stepq_pool *p)
 {
     if (!p) return;
@@ -310,6 +345,8 @@ int stepq_pool_load_fp32(stepq_pool *pool, const int32_t *slot_ids, int32_t n, c
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
     if (!S || !aligned16(S)) return STEPQ_INVALID_ARG;
+    st = debug_check_slots(pool, slot_ids, n, stream);
+    if (st != STEPQ_OK) return st;
     return status_of(stepq::launch_load_fp32(pool, slot_ids, n, S, stream));
 }
 
@@ -320,6 +357,8 @@ int stepq_pool_load_packed(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
     if (!bytes || !aligned16(bytes)) return STEPQ_INVALID_ARG;
+    st = debug_check_slots(pool, slot_ids, n, stream);
+    if (st != STEPQ_OK) return st;
     return status_of(stepq::launch_copy_slots(pool, slot_ids, n, bytes, nullptr, true, stream));
 }
 
@@ -330,6 +369,8 @@ int stepq_pool_dump_fp32(const stepq_pool *pool, const int32_t *slot_ids, int32_
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
     if (!S_out || !aligned16(S_out)) return STEPQ_INVALID_ARG;
+    st = debug_check_slots(pool, slot_ids, n, stream);
+    if (st != STEPQ_OK) return st;
     return status_of(stepq::launch_dump_fp32(pool, slot_ids, n, S_out, stream));
 }
 
@@ -340,6 +381,8 @@ int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot_ids, int3
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
     if (!bytes_out || !aligned16(bytes_out)) return STEPQ_INVALID_ARG;
+    st = debug_check_slots(pool, slot_ids, n, stream);
+    if (st != STEPQ_OK) return st;
     return status_of(stepq::launch_copy_slots(pool, slot_ids, n, nullptr, bytes_out, false, stream));
 }
 
@@ -355,6 +398,8 @@ int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, cons
     const size_t esz = pool->in_dtype == STEPQ_DTYPE_BF16 ? 2 : 4;
     if (pool->gate_mode == STEPQ_GATE_KDA ? !aligned16(alpha) : !aligned_to(alpha, esz)) return STEPQ_INVALID_ARG;
     if (!aligned_to(beta, esz)) return STEPQ_INVALID_ARG;
+    st = debug_check_slots(pool, slot_ids, n, stream);
+    if (st != STEPQ_OK) return st;
     return status_of(stepq::launch_decode(pool, slot_ids, n, q, k, v, alpha, beta, y, stream));
 }
 
@@ -366,6 +411,10 @@ int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
     if (!slot_ids || !q || !k || !v || !alpha || !beta || !y) return STEPQ_INVALID_ARG;
+    if (pool->debug & STEPQ_DEBUG_SLOTS) {
+        st = host_check_slot_ids(slot_ids, n, pool->num_slots);
+        if (st != STEPQ_OK) return st;
+    }
     const HostLayout L = host_layout(pool, n);
     st = host_prepare(pool, L.total);
     if (st != STEPQ_OK) return st;
@@ -437,6 +486,18 @@ int stepq_pool_set_impact(stepq_pool *pool, const float *impact)
     }
     e = cudaMemcpy(pool->d_impact, w.data(), sizeof(float) * size_t(n), cudaMemcpyHostToDevice);
     return status_of(e);
+}
+
+int stepq_pool_set_debug(stepq_pool *pool, int32_t flags)
+{
+    if (!pool || (flags & ~int32_t(STEPQ_DEBUG_SLOTS)) != 0) return STEPQ_INVALID_ARG;
+    pool->debug = flags;
+    return STEPQ_OK;
+}
+
+int stepq_check_slot_ids(const int32_t *slot_ids, int32_t n, int32_t num_slots)
+{
+    return host_check_slot_ids(slot_ids, n, num_slots);
 }
 
 int stepq_check_wait_timeout(int32_t *flag_out, stepq_stream stream)

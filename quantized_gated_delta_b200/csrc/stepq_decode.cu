@@ -1075,12 +1075,26 @@ constexpr int kNoallocFlagOffset = 0;                                     // int
 constexpr int kNoallocOffOffset = 256;                                    // int64[kMaxHeads]
 constexpr int kNoallocOrderOffset = kNoallocOffOffset + 8 * kMaxHeads;   // int32[kMaxHeads]
 constexpr int kNoallocBitsOffset = kNoallocOrderOffset + 4 * kMaxHeads;  // uint8[kMaxHeads]
-constexpr int kNoallocScratchBytes = kNoallocBitsOffset + kMaxHeads;      // 3328 bytes
+constexpr int kNoallocScratchBytes = kNoallocBitsOffset + kMaxHeads;      // 3584 bytes
+static_assert(kNoallocScratchBytes == 3584, "scratch size is documented in stepq.h");
 
 // Scratch of the allocation-free entry point.  Every GPU that loads the library holds it
 // until the process exits; host code reaches it only through the address returned by
 // cudaGetSymbolAddress (the symbol itself is a host-side stand-in).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+// The scratch contents of one call (flag word cleared, head tables), passed by value as the
+// argument of a one-CTA kernel that writes them into the array: no host memory is read by a
+// copy, so the call never waits on the host for earlier work of the stream.
+struct NoallocImage {
+    uint32_t words[kNoallocScratchBytes / 4];
+};
+
+__global__ void __launch_bounds__(256) noalloc_fill_kernel(const NoallocImage img)
+{
+    uint32_t *dst = reinterpret_cast<uint32_t *>(g_noalloc_scratch);
+    for (int i = threadIdx.x; i < kNoallocScratchBytes / 4; i += blockDim.x) dst[i] = img.words[i];
+}
 
 struct NoallocDevice {
     bool ready = false;
@@ -1173,8 +1187,9 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     NoallocDevice *nd = nullptr;
     if (noalloc_setup(dev, &nd) != cudaSuccess) return STEPQ_CUDA_ERROR;
 
-    // head tables (and a cleared flag word), staged in one host image of the scratch
-    alignas(16) uint8_t image[kNoallocScratchBytes] = {};
+    // head tables (and a cleared flag word) as one image of the scratch, written by a kernel
+    NoallocImage img = {};
+    uint8_t *image = reinterpret_cast<uint8_t *>(img.words);
     long long *off = reinterpret_cast<long long *>(image + kNoallocOffOffset);
     int32_t *order = reinterpret_cast<int32_t *>(image + kNoallocOrderOffset);
     uint8_t *bits = image + kNoallocBitsOffset;
@@ -1188,7 +1203,8 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
     for (int w = 4; w <= 8; w += 2)
         for (int h = 0; h < H; ++h)
             if (bits[h] == w) order[nord++] = h;
-    cudaError_t e = cudaMemcpyAsync(nd->scratch, image, kNoallocScratchBytes, cudaMemcpyHostToDevice, stream);
+    noalloc_fill_kernel<<<1, 256, 0, stream>>>(img);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return STEPQ_CUDA_ERROR;
 
     DecodeArgs a;

@@ -17,6 +17,7 @@ struct stepq_pool {
     int npiv = 0;                       // FP16 pivot heads (width 16), visited after the others
     int device = 0;
     int num_sms = 0;
+    int32_t debug = 0;                  // STEPQ_DEBUG_* flags (stepq_pool_set_debug)
     uint8_t *d_pool = nullptr;          // [num_slots * slot_stride]
     long long *d_offs = nullptr;        // [H]
     uint8_t *d_bits = nullptr;          // [H]

@@ -22,6 +22,7 @@ STEPQ_DTYPE_F32 = 0
 STEPQ_DTYPE_BF16 = 1
 STEPQ_FLAG_BAD_SLOT = 1
 STEPQ_FLAG_TIMEOUT = 2
+STEPQ_DEBUG_SLOTS = 1
 
 EXPORTED = [
     "stepq_pool_create", "stepq_pool_destroy", "stepq_pool_bytes", "stepq_pool_head_offset",
@@ -30,6 +31,7 @@ EXPORTED = [
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
     "stepq_allocate_bits_pivots", "stepq_pool_set_impact", "stepq_pool_create_rows",
     "stepq_check_wait_timeout", "stepq_decode_step_host", "stepq_pool_host_wait",
+    "stepq_pool_set_debug", "stepq_check_slot_ids",
 ]
 
 
@@ -76,6 +78,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_pool_host_wait": [P, P],
         "stepq_pool_create_rows": [ctypes.POINTER(stepq_pool_desc), P, ctypes.POINTER(P)],
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
+        "stepq_pool_set_debug": [P, I],
+        "stepq_check_slot_ids": [P, I, I],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -226,6 +230,16 @@ def stepq_pool_set_impact(pool: int, impact=None):
     _check(load_library().stepq_pool_set_impact(pool, w.ctypes.data), "stepq_pool_set_impact")
 
 
+def stepq_pool_set_debug(handle: int, flags: int) -> None:
+    _check(load_library().stepq_pool_set_debug(handle, int(flags)), "stepq_pool_set_debug")
+
+
+def stepq_check_slot_ids(slot_ids, num_slots: int) -> int:
+    """Status of the host-side slot-id check (0 when distinct and in range)."""
+    ids = np.ascontiguousarray(slot_ids, dtype=np.int32)
+    return load_library().stepq_check_slot_ids(ids.ctypes.data if ids.size else None, int(ids.size), int(num_slots))
+
+
 def stepq_check_wait_timeout(stream=None) -> int:
     """Run the kernels' bounded-wait failure path on a barrier nothing completes; returns the
     flag bits it raised (STEPQ_FLAG_TIMEOUT when the path works)."""
@@ -316,6 +330,9 @@ class Pool:
 
     def dump_packed(self, slot_ids, out, stream=None):
         stepq_pool_dump_packed(self.handle, slot_ids, out, stream)
+
+    def set_debug(self, flags: int) -> None:
+        stepq_pool_set_debug(self.handle, flags)
 
     def get_error(self) -> int:
         return stepq_pool_get_error(self.handle)
