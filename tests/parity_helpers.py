@@ -9,7 +9,7 @@ from quantized_gated_delta_b200 import workloads as W
 
 # Tolerances (the reading of the single-step bar; see the design notes):
 CODE_FLIP_RATE = 1e-5       # codes may differ by exactly 1 at this rate
-R_ULP = 8                   # row factors r within 8 ulp of the oracle's
+R_ULP = 6                   # row factors r within 6 ulp of the oracle's
 C_ULP = 4                   # column factors c within 4 ulp
 Y_MAX_REL = 1e-4            # per (request, head): max_j |dy_j| / max_j |y_j|
 Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
@@ -18,13 +18,14 @@ Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
 # oracle's double sums by at most ~(n-1) u, so c within 2e-5 relative.  An intermediate code
 # at a near tie may round one level apart (as any code may), which moves c_j by
 # w r^2 |P| / sum w r^2 Q0^2 -- a few percent in a column that a few rows carry; such columns
-# are counted like code flips and may be at most 1e-3 of the columns.  The codes follow c:
-# +-1 at a rate up to 1e-3.
+# are counted like code flips and may be at most 3e-4 of the columns (about 1e-4 seen over a
+# 256-step trajectory of the 512-request pool).  The codes follow c, yet even with those
+# columns the codes stay within the single-step bar of every other fit: +-1 at <= 1e-5.
 C_REL_IMPACT = 2e-5
-C_FAR_RATE_IMPACT = 1e-3
-CODE_FLIP_RATE_IMPACT = 1e-3
+C_FAR_RATE_IMPACT = 3e-4
+CODE_FLIP_RATE_IMPACT = 1e-5
 PIVOT_ULP = 1               # FP16 pivot states: binary16 values within 1 ulp ...
-PIVOT_FLIP_RATE = 1e-3      # ... and off by one ulp at most at this rate
+PIVOT_FLIP_RATE = 1e-4      # ... and off by one ulp at most at this rate (about 4e-5 seen)
 
 
 def head_bits(w: W.Workload, layer: int = 0) -> np.ndarray:

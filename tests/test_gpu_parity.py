@@ -547,6 +547,150 @@ def test_trajectory_parity(S, config, variant, batch, layer, nsample, steps):
     assert rel <= PH.Y_TRAJ_REL_L2
 
 
+# Free-running trajectories.  The per-step leg above re-synchronises a state whose codes came
+# out one level apart, so it checks each step from identical stored states.  Here nothing is
+# re-synchronised: the GPU runs the whole batch for the workload's full T, the oracle follows a
+# sample of requests with its own quantized state, and both are compared with the oracle's
+# unquantized (FP32-state) trajectory from the same starting state.  By the error recursion
+# of "Paper Explained: STEPQuant", "The intuition: errors get carried forward"
+# (E_t = A_t E_{t-1} + eps_t), the quantization error a trajectory accumulates is a property
+# of the quantizer, not of where the roundings fall; a GPU path that quantizes like the
+# oracle accumulates an error of the same size.  Bar: ||y_gpu - y_fp|| / ||y_oracle - y_fp||
+# in [FREE_BAND_LO, FREE_BAND_HI] over the sampled requests and all T steps (two correct
+# implementations of one quantizer land within a fraction of a percent of each other here).
+FREE_BAND_LO, FREE_BAND_HI = 0.95, 1.05
+
+FREE_CASES = [
+    # (config, variant, batch, layer, sampled requests)
+    (1, "mixed6", None, 0, 4),
+    (2, "mixed6", None, 0, 8),
+    (3, "mixed6", None, 0, 6),
+    (4, "mixed6", None, 0, 6),
+    (4, "uniform4", None, 0, 6),
+    (4, "mixed6p", None, 0, 6),
+    (3, "mixed6p", None, 0, 4),
+    (2, "mixed6p", None, 0, 6),
+    (3, "rowbits", None, 0, 4),
+    (5, "mixed6", 64, 17, 3),
+    (5, "mixed6", 1024, 35, 3),
+]
+
+
+@pytest.mark.parametrize("config,variant,batch,layer,nsample", FREE_CASES,
+                         ids=["cfg%d-%s-b%s-l%d" % (c[0], c[1], c[2], c[3]) for c in FREE_CASES])
+def test_free_running_trajectory(S, config, variant, batch, layer, nsample):
+    w = W.make_workload(config, variant, batch)
+    bits = PH.head_bits(w, layer)
+    sub = W.sample_requests(w, nsample)
+    sub_slots = w.slot_ids[sub]
+    op = PH.oracle_pool_with_warmup(w, bits, sub, layer)
+    rb = PH.row_bits(w, layer)
+    gp = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype, row_bits=rb)
+    load_bytes(gp, sub_slots, op.slot_bytes(sub_slots))
+    # the unquantized run starts from the same (dequantized) state
+    S_fp = op.dump_fp32(sub_slots).astype(np.float64)
+    all_slots = slots_t(w.slot_ids)
+    sub_t = torch.from_numpy(sub).cuda()
+    d_gpu = d_ora = d_go = n_ora = n_fp = 0.0
+    for t in range(w.T):
+        x = W.step_inputs(w, t, W.PHASE_RUN, layer)
+        tx = PH.to_device(w, x, torch)
+        y = torch.empty((w.B, w.H, w.dv), device="cuda")
+        gp.decode_step(all_slots, tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        xs = PH.sub_inputs(x, sub)
+        yo = op.decode_step(sub_slots, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"]).astype(np.float64)
+        yf = O.fp_decode_step(S_fp, w.Hk, w.gate_mode, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"],
+                              round_fp32=True).astype(np.float64)
+        yg = y[sub_t].cpu().numpy().astype(np.float64)
+        d_gpu += float(np.sum((yg - yf) ** 2))
+        d_ora += float(np.sum((yo - yf) ** 2))
+        d_go += float(np.sum((yg - yo) ** 2))
+        n_ora += float(np.sum(yo ** 2))
+        n_fp += float(np.sum(yf ** 2))
+    assert gp.get_error() == 0
+    ratio = np.sqrt(d_gpu / d_ora)
+    print("\n%s free-running T=%d: quantization error vs FP32 state: gpu %.3e, oracle %.3e (ratio %.4f); "
+          "gpu vs oracle y rel L2 %.3e" % (w.name, w.T, np.sqrt(d_gpu / n_fp), np.sqrt(d_ora / n_fp), ratio,
+                                          np.sqrt(d_go / n_ora)))
+    assert FREE_BAND_LO <= ratio <= FREE_BAND_HI
+
+
+# --------------------------------------------------------------------------- checkpoint and debug mode
+
+def test_checkpoint_restore_continues_bit_identically(S):
+    """Dump a pool's packed slots after a few steps, restore them into a fresh pool with
+    load_packed, and continue both pools with the same inputs: y and the packed states stay
+    bit-identical (the pool layout is the whole state of a request)."""
+    w = W.make_workload(4, "mixed6p")
+    bits = PH.head_bits(w)
+    n = 64
+    ids = w.slot_ids[:n]
+    rng = np.random.default_rng(404)
+    S0 = random_states(rng, n, w.H, steps=16)
+    a = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    a.load_fp32(slots_t(ids), dev(S0))
+    xs = []
+    for t in range(12):
+        x = PH.sub_inputs(W.step_inputs(w, t), np.arange(n))
+        xs.append(PH.to_device(w, x, torch))
+    y = torch.empty((n, w.H, w.dv), device="cuda")
+    for t in range(4):
+        a.decode_step(slots_t(ids), xs[t]["q"], xs[t]["k"], xs[t]["v"], xs[t]["alpha"], xs[t]["beta"], y)
+    ckpt = dump_bytes(a, ids)
+    b = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    load_bytes(b, ids, ckpt)
+    ya = torch.empty_like(y)
+    yb = torch.empty_like(y)
+    for t in range(4, 12):
+        a.decode_step(slots_t(ids), xs[t]["q"], xs[t]["k"], xs[t]["v"], xs[t]["alpha"], xs[t]["beta"], ya)
+        b.decode_step(slots_t(ids), xs[t]["q"], xs[t]["k"], xs[t]["v"], xs[t]["alpha"], xs[t]["beta"], yb)
+        torch.cuda.synchronize()
+        assert torch.equal(ya, yb)
+    assert np.array_equal(dump_bytes(a, ids), dump_bytes(b, ids))
+    assert a.get_error() == 0 and b.get_error() == 0
+    a.close()
+    b.close()
+
+
+def test_debug_mode_rejects_duplicate_slot_ids(S):
+    """With STEPQ_DEBUG_SLOTS a step with a repeated or out-of-range slot id is refused before
+    any device work (the states stay as they were); distinct ids give the same step as
+    without the debug mode."""
+    bits = np.array([4, 6, 8, 16], np.int32)
+    rng = np.random.default_rng(5)
+    n, H, Hk = 4, 4, 2
+    S0 = random_states(rng, n, H)
+    ids = np.array([5, 1, 6, 2], np.int32)
+    pools = [S.Pool(8, bits, Hk, 0, 0) for _ in range(2)]
+    for p in pools:
+        p.load_fp32(slots_t(ids), dev(S0))
+    pools[1].set_debug(S.STEPQ_DEBUG_SLOTS)
+    x = dict(q=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
+             k=np.stack([[unit(rng, 128) for _ in range(Hk)] for _ in range(n)]),
+             v=rng.standard_normal((n, H, 128)).astype(f32), alpha=np.full((n, H), 0.9, f32),
+             beta=np.full((n, H), 0.5, f32))
+    tx = {k_: dev(v_) for k_, v_ in x.items()}
+    y = torch.zeros((n, H, 128), device="cuda")
+    before = dump_bytes(pools[1], ids)
+    for bad in ([5, 1, 5, 2], [5, 1, 8, 2], [5, -1, 6, 2]):
+        with pytest.raises(S.StepqError) as err:
+            pools[1].decode_step(slots_t(bad), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        assert err.value.status == -1
+    assert np.array_equal(dump_bytes(pools[1], ids), before)
+    assert float(y.abs().max()) == 0.0
+    ys = []
+    for p in pools:
+        yp = torch.empty((n, H, 128), device="cuda")
+        p.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], yp)
+        torch.cuda.synchronize()
+        ys.append(yp.cpu().numpy())
+    assert np.array_equal(ys[0], ys[1])
+    assert np.array_equal(dump_bytes(pools[0], ids), dump_bytes(pools[1], ids))
+    for p in pools:
+        assert p.get_error() == 0
+        p.close()
+
+
 # --------------------------------------------------------------------------- impact-weighted fit
 
 def _impact_scores(rng, H):
