@@ -354,6 +354,9 @@ def run_stack(args):
             raise RuntimeError("device flag set in the stack sweep")
     units = w.B * w.H * L * args.steps
     value = units / (ms_graph / 1e3)
+    # the same pool with FP32 states (d_k x d_v float32 per head, no scales): the pages'
+    # reference point for the state-pool memory
+    fp32_bytes = int(L * w.num_slots * w.H * w.dk * w.dv * 4)
     alg = sum(algorithmic_bytes_per_step(w, b) for b in bits_all)          # one step, all layers
     peak, peak_kind = peaks()
     achieved = alg * args.steps / (ms_graph / 1e3) / 1e9
@@ -364,6 +367,8 @@ def run_stack(args):
             "config": {"workload": "%s: %d layers x H=%d, Hk=%d, B=%d, per-layer allocation (6.0 avg), bf16 inputs"
                                    % (w.name, L, w.H, w.Hk, w.B),
                        "pool_bytes": int(sum(p_.total_bytes for p_ in pools)),
+                       "fp32_pool_bytes": fp32_bytes,
+                       "fp32_over_packed": fp32_bytes / float(sum(p_.total_bytes for p_ in pools)),
                        "l2": "no flush: each layer's pool is re-read after the other 35 (stack > 126 MB L2)"},
             "us_per_layer_step_graph": ms_graph * 1e3 / (args.steps * L),
             "us_per_layer_step_plain": ms_plain * 1e3 / (args.steps * L),

@@ -179,6 +179,15 @@ STEPQ_API int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, 
                                      const void *k, const void *v, const void *alpha, const void *beta, float *y,
                                      stepq_stream stream);
 
+/* Layout of a contiguous host input image for stepq_decode_step_host: for n requests of this
+ * pool, offsets_out[0..5] (HOST, 6 entries) receive the byte offsets of slot_ids, q, k, v,
+ * alpha and beta from the start of the image (slot_ids at 0, each a multiple of 256 bytes,
+ * each array as laid out for stepq_decode_step), and total_out (may be NULL) the image's
+ * size.  When a call's six host inputs sit at exactly these offsets of one buffer (slot_ids
+ * at its start), the call copies them to the device as one transfer instead of six; any
+ * other placement works as before.  The paper has no counterpart. */
+STEPQ_API int stepq_host_image_layout(const stepq_pool *pool, int32_t n, size_t *offsets_out, size_t *total_out);
+
 /* Makes `stream` wait for every copy that stepq_decode_step_host calls on this pool have
  * enqueued, y included.  Enqueues only; synchronize `stream` to wait on the host. */
 STEPQ_API int stepq_pool_host_wait(stepq_pool *pool, stepq_stream stream);

@@ -421,14 +421,22 @@ int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
     const int b = int(pool->host_calls & 1);
     uint8_t *d = pool->d_host_stage[b];
     const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+    // inputs laid out as one contiguous image (stepq_host_image_layout) go in one copy
+    const uint8_t *img = reinterpret_cast<const uint8_t *>(slot_ids);
+    const bool one_image = q == img + L.q && k == img + L.k && v == img + L.v && alpha == img + L.alpha &&
+                           beta == img + L.beta;
     // copy-in, once the step that last read this staging buffer is done
     cudaError_t e = cudaStreamWaitEvent(pool->s_in, pool->ev_step[b], 0);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.slots, slot_ids, size_t(n) * 4, h2d, pool->s_in);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.q, q, L.qk_bytes, h2d, pool->s_in);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.k, k, L.qk_bytes, h2d, pool->s_in);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.v, v, L.v_bytes, h2d, pool->s_in);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.alpha, alpha, L.alpha_bytes, h2d, pool->s_in);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.beta, beta, L.beta_bytes, h2d, pool->s_in);
+    if (one_image) {
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d, img, L.beta + L.beta_bytes, h2d, pool->s_in);
+    } else {
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.slots, slot_ids, size_t(n) * 4, h2d, pool->s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.q, q, L.qk_bytes, h2d, pool->s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.k, k, L.qk_bytes, h2d, pool->s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.v, v, L.v_bytes, h2d, pool->s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.alpha, alpha, L.alpha_bytes, h2d, pool->s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(d + L.beta, beta, L.beta_bytes, h2d, pool->s_in);
+    }
     if (e == cudaSuccess) e = cudaEventRecord(pool->ev_in[b], pool->s_in);
     // the step on the caller's stream, once its inputs are in and the copy-out that last read
     // this buffer's y is done
@@ -444,6 +452,16 @@ int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
     if (e == cudaSuccess) e = cudaEventRecord(pool->ev_out[b], pool->s_out);
     ++pool->host_calls;
     return status_of(e);
+}
+
+int stepq_host_image_layout(const stepq_pool *pool, int32_t n, size_t *offsets_out, size_t *total_out)
+{
+    if (!pool || !offsets_out || n < 0 || n > pool->num_slots || n > 65535) return STEPQ_INVALID_ARG;
+    const HostLayout L = host_layout(pool, n);
+    const size_t o[6] = {L.slots, L.q, L.k, L.v, L.alpha, L.beta};
+    for (int i = 0; i < 6; ++i) offsets_out[i] = o[i];
+    if (total_out) *total_out = L.beta + L.beta_bytes;
+    return STEPQ_OK;
 }
 
 int stepq_pool_host_wait(stepq_pool *pool, stepq_stream stream)

@@ -31,7 +31,7 @@ EXPORTED = [
     "stepq_allocate_bits", "stepq_status_string", "stepq_decode_step_noalloc",
     "stepq_allocate_bits_pivots", "stepq_pool_set_impact", "stepq_pool_create_rows",
     "stepq_check_wait_timeout", "stepq_decode_step_host", "stepq_pool_host_wait",
-    "stepq_pool_set_debug", "stepq_check_slot_ids",
+    "stepq_pool_set_debug", "stepq_check_slot_ids", "stepq_host_image_layout",
 ]
 
 
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "stepq_decode_step_noalloc": [ctypes.POINTER(stepq_pool_desc), P, P, I, P, P, P, P, P, P, P, P],
         "stepq_pool_set_debug": [P, I],
         "stepq_check_slot_ids": [P, I, I],
+        "stepq_host_image_layout": [P, I, P, ctypes.POINTER(Z)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -240,6 +241,16 @@ def stepq_check_slot_ids(slot_ids, num_slots: int) -> int:
     return load_library().stepq_check_slot_ids(ids.ctypes.data if ids.size else None, int(ids.size), int(num_slots))
 
 
+def stepq_host_image_layout(handle: int, n: int):
+    """(offsets of slot_ids, q, k, v, alpha, beta; total bytes) of the contiguous host input
+    image of n requests."""
+    offs = (ctypes.c_size_t * 6)()
+    total = ctypes.c_size_t()
+    _check(load_library().stepq_host_image_layout(handle, int(n), offs, ctypes.byref(total)),
+           "stepq_host_image_layout")
+    return [int(o) for o in offs], int(total.value)
+
+
 def stepq_check_wait_timeout(stream=None) -> int:
     """Run the kernels' bounded-wait failure path on a barrier nothing completes; returns the
     flag bits it raised (STEPQ_FLAG_TIMEOUT when the path works)."""
@@ -330,6 +341,9 @@ class Pool:
 
     def dump_packed(self, slot_ids, out, stream=None):
         stepq_pool_dump_packed(self.handle, slot_ids, out, stream)
+
+    def host_image_layout(self, n: int):
+        return stepq_host_image_layout(self.handle, n)
 
     def set_debug(self, flags: int) -> None:
         stepq_pool_set_debug(self.handle, flags)

@@ -33,6 +33,7 @@ int fail_handle_at = -1;
 std::set<void *> live;         // fake device allocations not yet freed
 std::set<void *> handles;      // live streams and events
 int launches = 0;
+int h2d_copies = 0;            // cudaMemcpyAsync calls from host to device
 const int32_t *last_slots = nullptr;
 int last_n = 0;
 const void *last_q = nullptr;
@@ -120,8 +121,9 @@ cudaError_t cudaMemcpy(void *d, const void *s, size_t n, cudaMemcpyKind)
     std::memcpy(d, s, n);
     return cudaSuccess;
 }
-cudaError_t cudaMemcpyAsync(void *d, const void *s, size_t n, cudaMemcpyKind, cudaStream_t)
+cudaError_t cudaMemcpyAsync(void *d, const void *s, size_t n, cudaMemcpyKind kind, cudaStream_t)
 {
+    if (kind == cudaMemcpyHostToDevice) ++fake::h2d_copies;
     std::memcpy(d, s, n);
     return cudaSuccess;
 }
@@ -390,6 +392,34 @@ static void test_host_path_staging()
         CHECK(reinterpret_cast<const uint8_t *>(fake::last_q) > stage &&
               reinterpret_cast<const uint8_t *>(fake::last_q) < stage + p->host_stage_cap);
     }
+    // inputs placed at the offsets of stepq_host_image_layout: one host-to-device copy, same data
+    for (int n : {1, 9, 64}) {
+        size_t off[6] = {0}, total = 0;
+        CHECK(stepq_host_image_layout(p, n, off, &total) == STEPQ_OK);
+        CHECK(off[0] == 0 && total > off[5]);
+        for (int i = 1; i < 6; ++i) CHECK(off[i] % 256 == 0 && off[i] > off[i - 1]);
+        std::vector<uint8_t> image(total, 0);
+        int32_t *ids = reinterpret_cast<int32_t *>(image.data());
+        for (int i = 0; i < n; ++i) ids[i] = (5 * i + 3) % 64;
+        for (size_t e = off[1]; e < total; ++e) image[e] = uint8_t(e * 7 + n);
+        std::vector<float> y(size_t(n) * 4 * 128);
+        const uint8_t *I = image.data();
+        const int before = fake::h2d_copies;
+        CHECK(stepq_decode_step_host(p, ids, n, I + off[1], I + off[2], I + off[3], I + off[4], I + off[5],
+                                     y.data(), nullptr) == STEPQ_OK);
+        CHECK(fake::h2d_copies == before + 1);
+        CHECK(std::memcmp(fake::last_slots, ids, sizeof(int32_t) * n) == 0);
+        CHECK(std::memcmp(fake::last_q, I + off[1], off[2] - off[1]) == 0);
+        // one array elsewhere: six copies
+        std::vector<uint8_t> other(I + off[3], I + off[4]);
+        const int before6 = fake::h2d_copies;
+        CHECK(stepq_decode_step_host(p, ids, n, I + off[1], I + off[2], other.data(), I + off[4], I + off[5],
+                                     y.data(), nullptr) == STEPQ_OK);
+        CHECK(fake::h2d_copies == before6 + 6);
+    }
+    size_t off[6];
+    CHECK(stepq_host_image_layout(p, 65, off, nullptr) == STEPQ_INVALID_ARG);
+    CHECK(stepq_host_image_layout(p, 2, nullptr, nullptr) == STEPQ_INVALID_ARG);
     CHECK(stepq_pool_host_wait(p, nullptr) == STEPQ_OK);
     CHECK(stepq_pool_destroy(p) == STEPQ_OK);
     CHECK(fake::live.empty() && fake::handles.empty());
