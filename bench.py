@@ -504,17 +504,28 @@ def main():
     # ---- end-to-end leg: the host-buffer entry point.  Slot ids, inputs and y live in pinned
     # host memory; every step the library copies that step's inputs in and its y out, through
     # two staging buffers, so the copies of one step overlap the neighbouring steps' kernels.
+    # each step's slot ids and inputs sit in one pinned image at the offsets the library gives
+    # (stepq_host_image_layout), so the call copies them in one transfer
+    offs, img_bytes = pool.host_image_layout(w.B)
+    names = ("slots", "q", "k", "v", "alpha", "beta")
     host = []
     for x in host_sets[:E2E_HOST_SETS]:
-        host.append({k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).pin_memory() for k, v in x.items()})
+        img = torch.zeros(img_bytes, dtype=torch.uint8).pin_memory()
+        arrays = [np.ascontiguousarray(w.slot_ids, dtype=np.int32)] + \
+                 [W.as_device_dtype(w, x[k]).view(np.int16) for k in names[1:]]
+        views = {}
+        for name, o, a in zip(names, offs, arrays):
+            t = torch.from_numpy(a.reshape(-1))
+            img[o:o + t.numel() * t.element_size()].copy_(t.view(torch.uint8))
+            views[name] = img[o:o + t.numel() * t.element_size()].view(t.dtype)
+        host.append(views)
     y_host = torch.empty((w.B, w.H, w.dv), dtype=torch.float32).pin_memory()
-    slots_host = torch.from_numpy(w.slot_ids).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host[0].values()) + slots_host.numel() * 4
+    h2d = img_bytes
     d2h = y_host.numel() * 4
 
     def e2e_step(i):
         hx = host[i % len(host)]
-        pool.decode_step_host(slots_host, hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], y_host, stream)
+        pool.decode_step_host(hx["slots"], hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], y_host, stream)
 
     for i in range(3):
         e2e_step(i)
@@ -550,7 +561,9 @@ def main():
                          "kernel": "decode_kernel", "avg_kernel_us": avg_kernel_s * 1e6},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps,
-                    "api": "stepq_decode_step_host: pinned host buffers, copies of consecutive steps overlapped"},
+                    "api": "stepq_decode_step_host: one pinned input image per step (stepq_host_image_layout), "
+                           "one host-to-device and one device-to-host copy per step, copies of consecutive steps "
+                           "overlapped"},
             "timing": ("device leg: %d-step CUDA-graph chunks replayed" % graphed if graphed else
                        "device leg: plain launches (graph capture failed: %s)" % capture_error)
                       + " (kernel time = region / steps); plain launches with one event pair each: %.1f us median"

@@ -19,13 +19,14 @@ Y_TRAJ_REL_L2 = 1e-3        # whole trajectory: ||dy||_2 / ||y||_2
 # at a near tie may round one level apart (as any code may), which moves c_j by
 # w r^2 |P| / sum w r^2 Q0^2 -- a few percent in a column that a few rows carry; such columns
 # are counted like code flips and may be at most 3e-4 of the columns (about 1e-4 seen over a
-# 256-step trajectory of the 512-request pool).  The codes follow c, yet even with those
-# columns the codes stay within the single-step bar of every other fit: +-1 at <= 1e-5.
+# 256-step trajectory of the 512-request pool).  The codes of such a column follow its c and
+# are not held to a flip rate; in every other column codes are +-1 at <= 1e-5, the
+# single-step bar of the clip-free fit (1.3e-6 seen).
 C_REL_IMPACT = 2e-5
 C_FAR_RATE_IMPACT = 3e-4
 CODE_FLIP_RATE_IMPACT = 1e-5
 PIVOT_ULP = 1               # FP16 pivot states: binary16 values within 1 ulp ...
-PIVOT_FLIP_RATE = 1e-4      # ... and off by one ulp at most at this rate (about 4e-5 seen)
+PIVOT_FLIP_RATE = 1e-3      # ... and off by one ulp at most at this rate (see pivots_ok)
 
 
 def head_bits(w: W.Workload, layer: int = 0) -> np.ndarray:
@@ -169,10 +170,15 @@ def compare_slots(gpu_bytes: np.ndarray, ora_bytes: np.ndarray, bits, dk=128, dv
             res["r_ulp"] = max(res["r_ulp"], int(ulp_diff(rg, ro).max()))
             res["c_ulp"] = max(res["c_ulp"], int(ulp_diff(cg, co).max()))
             nz = co != 0
-            rel = np.abs(cg[nz].astype(np.float64) - co[nz]) / np.abs(co[nz]) if nz.any() else np.zeros(1)
+            rel_all = np.zeros(co.shape)
+            rel_all[nz] = np.abs(cg[nz].astype(np.float64) - co[nz]) / np.abs(co[nz])
+            rel = rel_all[nz] if nz.any() else np.zeros(1)
             res["c_rel"] = max(res.get("c_rel", 0.0), float(rel.max()))
             res["c_far"] = res.get("c_far", 0) + int(np.sum(rel > C_REL_IMPACT))
             res["c_cols"] = res.get("c_cols", 0) + int(cg.size)
+            # code flips outside the columns whose scale moved (impact fit, see C_FAR_RATE_IMPACT)
+            near = rel_all <= C_REL_IMPACT
+            res["flips_near"] = res.get("flips_near", 0) + int(((d > 0) & near[None, :]).sum())
             res["zero_c_mismatch"] = res.get("zero_c_mismatch", 0) + int(np.sum((co == 0) != (cg == 0)))
     return res
 
@@ -187,7 +193,11 @@ def y_max_rel(yg: np.ndarray, yo: np.ndarray) -> float:
 
 def pivots_ok(res: dict) -> bool:
     """The FP16 pivot bar: every binary16 value within PIVOT_ULP, off-by-one at a rate of at
-    most PIVOT_FLIP_RATE (fp32 kernel arithmetic against the fp64 oracle before rounding)."""
+    most PIVOT_FLIP_RATE.  The kernel rounds an fp32-computed value to binary16, the oracle its
+    fp64 value (to fp32, then binary16): they part only where the value lies within the fp32
+    error of a binary16 rounding boundary, a share of about 2^-12 k of the values for an error
+    of k fp32 ulps (k up to ~4 where the fade and the write nearly cancel).  Trajectories show
+    3-4e-5; single steps from fresh random states more."""
     if res["pivot_elements"] == 0:
         return True
     return res["pivot_ulp"] <= PIVOT_ULP and res["pivot_flips"] <= max(1, PIVOT_FLIP_RATE * res["pivot_elements"])

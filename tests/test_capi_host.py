@@ -132,3 +132,42 @@ def test_vectorised_dp_equals_library_allocator_at_row_granularity(S):
     got = S.stepq_allocate_bits(hl, None, (4, 6, 8), 6.0)
     assert list(got) == ref
     assert got.mean() == 6.0
+
+
+def test_allocation_from_measured_distortions(S):
+    """The allocator fed with measured reconstruction distortions ([SUM] Method para 2:
+    'estimate the reconstruction distortion at various bit widths'): D_u(b) = mean over
+    requests of ||S - deq(Q_b(S))||_F^2 on FP32 warm-up states of the hybrid GDN layer,
+    measured with the oracle's clip-free quantizer.  The library's C++ allocator equals the
+    oracle's DP on that table, every distortion falls with the width, and the measured ratios
+    sit near the uniform quantizer's 2^(-2 b) power law that the workloads use when no table
+    is given (one step of width, 2 bits, divides the error power by ~16)."""
+    from quantized_gated_delta_b200 import workloads as W
+    w = W.make_workload(2)
+    req = np.arange(4)
+    Sd = np.zeros((len(req), w.H, 128, 128))
+    for t in range(w.warmup_steps):
+        x = {k: np.ascontiguousarray(v[req]) for k, v in W.step_inputs(w, t, W.PHASE_WARMUP).items()}
+        O.fp_decode_step(Sd, w.Hk, w.gate_mode, x["q"], x["k"], x["v"], x["alpha"], x["beta"], round_fp32=True)
+    S32 = Sd.astype(np.float32)
+    cand = [4, 6, 8]
+    D = np.zeros((w.H, len(cand)))
+    for h in range(w.H):
+        for ci, b in enumerate(cand):
+            err = 0.0
+            for r in range(len(req)):
+                Q, rr, cc = O.quantize(S32[r, h], b)[:3]
+                err += float(np.sum((S32[r, h].astype(np.float64) - O.dequantize(Q, rr, cc)) ** 2))
+            D[h, ci] = err / len(req)
+    assert np.all(D[:, 0] > D[:, 1]) and np.all(D[:, 1] > D[:, 2])
+    ratio = np.concatenate([D[:, 0] / D[:, 1], D[:, 1] / D[:, 2]])
+    assert 14.0 < np.median(ratio) < 24.0            # 18.2 measured
+    hl = w.half_life[0]
+    ref, _ = O.allocate_bits_dp(list(hl), D, cand, w.avg_bits)
+    got = S.stepq_allocate_bits(hl, D, (4, 6, 8), w.avg_bits)
+    assert list(got) == ref and got.mean() == w.avg_bits
+    # on this layer the measured table picks exactly the widths of the power-law model (the
+    # measured ratio per 2 bits is ~18 against the model's 16, and the distortion spread
+    # between heads is small next to their lifetime weights, which span three decades)
+    model = S.stepq_allocate_bits(hl, None, (4, 6, 8), w.avg_bits)
+    assert list(got) == list(model)

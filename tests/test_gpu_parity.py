@@ -235,7 +235,7 @@ def test_pivot_heads_load_dump_and_step(S):
         yo = op2.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
         assert err == 0
         res = PH.compare_slots(sg, op2.slot_bytes(ids), bits)
-        assert PH.pivots_ok(res), res
+        assert PH.pivots_ok(res), (res["pivot_flips"], res["pivot_elements"], res["pivot_ulp"])
         assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
         assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
 
@@ -263,7 +263,7 @@ def test_max_heads_vs_oracle(S):
     assert err == 0
     yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
     res = PH.compare_slots(sg, op.slot_bytes(ids), bits)
-    assert PH.pivots_ok(res), res
+    assert PH.pivots_ok(res), (res["pivot_flips"], res["pivot_elements"], res["pivot_ulp"])
     assert res["max_code_diff"] <= 1 and res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
     assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
     assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
@@ -401,8 +401,9 @@ def test_host_buffer_steps_match_device_steps(S, gate, dtype):
     """stepq_decode_step_host (slot ids, inputs and y in host memory; copy-in, step and
     copy-out of consecutive calls overlapped through two staging buffers) gives outputs and
     states bit-identical to stepq_decode_step on device buffers, call after call: six calls
-    enqueued back to back on pinned buffers, then one on pageable buffers, then a larger
-    batch that regrows the staging buffers.  GDN with bf16 inputs and KDA (per-channel gate
+    enqueued back to back on pinned buffers (three with separate arrays, three with one
+    contiguous input image copied in one transfer), then one on pageable buffers, then a
+    larger batch that regrows the staging buffers.  GDN with bf16 inputs and KDA (per-channel gate
     vectors in the staging buffer) with fp32 inputs."""
     rng = np.random.default_rng(5)
     bits, H, Hk, num_slots = [4, 6, 8, 6], 4, 2, 12
@@ -422,20 +423,36 @@ def test_host_buffer_steps_match_device_steps(S, gate, dtype):
             return {key: torch.from_numpy(val) for key, val in x.items()}
         return {key: torch.from_numpy(W.to_bf16_bits(val).view(np.int16)) for key, val in x.items()}
 
-    plan = [(5, True)] * 6 + [(5, False), (8, True)]
-    steps = [(ids_all[:n], inputs(n), pinned) for n, pinned in plan]
+    # "pinned": six pinned arrays; "image": one pinned image at the offsets of
+    # stepq_host_image_layout (one copy-in); "pageable": ordinary host memory
+    plan = [(5, "pinned")] * 3 + [(5, "image")] * 3 + [(5, "pageable"), (8, "image")]
+    steps = [(ids_all[:n], inputs(n), mode) for n, mode in plan]
     y_dev = []
     for ids, x, _ in steps:
         y = torch.empty((len(ids), H, 128), device="cuda")
         pools[0].decode_step(slots_t(ids), *[x[key].cuda() for key in ("q", "k", "v", "alpha", "beta")], y)
         y_dev.append(y.cpu().numpy())
     y_host = []
-    for ids, x, pinned in steps:
-        hx = {key: (val.pin_memory() if pinned else val.clone()) for key, val in x.items()}
+    for ids, x, mode in steps:
         hs = torch.from_numpy(ids.copy())
         yh = torch.full((len(ids), H, 128), float("nan"))
-        if pinned:
-            hs, yh = hs.pin_memory(), yh.pin_memory()
+        if mode == "image":
+            offs, total = pools[1].host_image_layout(len(ids))
+            img = torch.zeros(total, dtype=torch.uint8).pin_memory()
+            hx = {}
+            for name, o, t in zip(("slots", "q", "k", "v", "alpha", "beta"), offs,
+                                  [hs] + [x[key] for key in ("q", "k", "v", "alpha", "beta")]):
+                nb = t.numel() * t.element_size()
+                img[o:o + nb].copy_(t.reshape(-1).view(torch.uint8))
+                hx[name] = img[o:o + nb].view(t.dtype)
+            hs = hx.pop("slots")
+            hx["image"] = img
+            yh = yh.pin_memory()
+        else:
+            pinned = mode == "pinned"
+            hx = {key: (val.pin_memory() if pinned else val.clone()) for key, val in x.items()}
+            if pinned:
+                hs, yh = hs.pin_memory(), yh.pin_memory()
         pools[1].decode_step_host(hs, hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], yh)
         y_host.append((yh, hx, hs))                 # keep the host buffers alive until the wait
     pools[1].host_wait()
@@ -716,7 +733,7 @@ def test_impact_fit_load_and_step_vs_oracle(S):
     res = PH.compare_slots(dump_bytes(gp, ids), op.slot_bytes(ids), bits)
     assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP
     assert PH.impact_scales_ok(res), res
-    assert res["flips"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"])
+    assert res["flips_near"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"]), res
     for gate, dtype, Hk in ((0, S.STEPQ_DTYPE_F32, H), (1, S.STEPQ_DTYPE_BF16, 2)):
         op2 = O.OraclePool(3, bits, Hk, gate, impact=omega)
         op2.load_fp32(ids, st)
@@ -738,7 +755,7 @@ def test_impact_fit_load_and_step_vs_oracle(S):
         res = PH.compare_slots(dump_bytes(gp2, ids), op2.slot_bytes(ids), bits)
         assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP, res
         assert PH.impact_scales_ok(res), res
-        assert res["flips"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"]), res
+        assert res["flips_near"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"]), res
         assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL
 
 
