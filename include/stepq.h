@@ -253,7 +253,7 @@ STEPQ_API int stepq_pool_set_debug(stepq_pool *pool, int32_t flags);
 
 /* The same check on a HOST array: STEPQ_OK when slot_ids[0 .. n) are distinct and each lies in
  * [0, num_slots), else STEPQ_INVALID_ARG (also for n < 0, num_slots <= 0, or a null array
- * with n > 0). */
+ * with n > 0).  Reads the array only; no device work.  The paper has no counterpart. */
 STEPQ_API int stepq_check_slot_ids(const int32_t *slot_ids, int32_t n, int32_t num_slots);
 
 /* Read and clear the pool's sticky device flag (host output, STEPQ_FLAG_* bits).
