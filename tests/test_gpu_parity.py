@@ -321,6 +321,33 @@ def _run_gpu(S, bits, Hk, gate, dtype, x, init_bytes, ids, num_slots):
     return y.cpu().numpy(), dump_bytes(gp, ids), gp.get_error()
 
 
+@pytest.mark.parametrize("H,Hk,gate,n", [(8, 2, 0, 37), (16, 1, 1, 5), (32, 4, 0, 19)],
+                         ids=["group4-gdn-n37", "group16-kda-n5", "group8-gdn-n19"])
+def test_key_head_groups_vs_oracle(S, H, Hk, gate, n):
+    """Value heads sharing one key head in groups of 4, 8 and 16 (consecutive grouping,
+    g(h) = h / (H / Hk)), every width and an FP16 pivot head, a batch size that fills no
+    whole number of CTA passes, one step against the oracle with the single-step bars."""
+    rng = np.random.default_rng(100 + H + Hk)
+    bits = [(4, 6, 8, 16, 6, 4, 8, 6)[h % 8] for h in range(H)]
+    num_slots = n + 3
+    ids = rng.permutation(num_slots)[:n].astype(np.int32)
+    st = random_states(rng, n, H, steps=6)
+    op = O.OraclePool(num_slots, bits, Hk, gate)
+    op.load_fp32(ids, st)
+    x = dict(q=_unit_rows(rng, (n, Hk)), k=_unit_rows(rng, (n, Hk)),
+             v=rng.standard_normal((n, H, 128)).astype(f32),
+             alpha=rng.uniform(0.7, 1, (n, H) if gate == 0 else (n, H, 128)).astype(f32),
+             beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+    yg, sg, err = _run_gpu(S, bits, Hk, gate, S.STEPQ_DTYPE_F32, x, op.slot_bytes(ids), ids, num_slots)
+    assert err == 0
+    yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    res = PH.compare_slots(sg, op.slot_bytes(ids), bits)
+    assert PH.pivots_ok(res), (res["pivot_flips"], res["pivot_elements"], res["pivot_ulp"])
+    assert res["max_code_diff"] <= 1 and res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
+    assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP
+    assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
+
+
 def test_kda_equal_gates_gqa_and_bf16_identities(S):
     """Bit identities on the GPU: KDA with equal per-channel gates = GDN; Hk = 2 with
     H = 4 = repeated key heads; bf16 inputs = the same values given as fp32."""
@@ -856,3 +883,46 @@ def test_rowbits_heads_load_dump_and_step(S):
     assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP, res
     assert res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"])
     assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL
+
+
+def test_rowbits_and_impact_fit_in_one_pool(S):
+    """A pool with per-key-row heads next to uniform heads and row-impact scores set: the
+    uniform heads take the impact-weighted fit, the per-row heads keep the clip-free fit at
+    each row's levels (both fit options in one kernel).  One KDA bf16 step against the oracle:
+    the impact bars on the uniform heads, the single-step bars on the per-row heads."""
+    rng = np.random.default_rng(16)
+    H, n = 4, 3
+    bits = [0, 8, 0, 6]
+    rb = np.stack([rng.choice([4, 6, 8], 128, p=[0.4, 0.4, 0.2]) for _ in range(H)]).astype(np.int32)
+    omega = _impact_scores(rng, H)
+    st = random_states(rng, n, H)
+    ids = np.array([2, 0, 3], np.int32)
+    op = O.OraclePool(4, bits, 2, 1, row_bits=rb, impact=omega)
+    op.load_fp32(ids, st)
+    gp = S.Pool(4, bits, 2, S.STEPQ_GATE_KDA, S.STEPQ_DTYPE_BF16, row_bits=rb)
+    gp.set_impact(omega)
+    load_bytes(gp, ids, op.slot_bytes(ids))
+    x = dict(q=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)])),
+             k=W.round_bf16(np.stack([[unit(rng, 128) for _ in range(2)] for _ in range(n)])),
+             v=W.round_bf16(rng.standard_normal((n, H, 128)).astype(f32)),
+             alpha=W.round_bf16(rng.uniform(0.6, 1, (n, H, 128)).astype(f32)),
+             beta=W.round_bf16(rng.uniform(0.1, 0.9, (n, H)).astype(f32)))
+    tx = {k_: dev(W.to_bf16_bits(v_).view(np.int16)) for k_, v_ in x.items()}
+    y = torch.empty((n, H, 128), device="cuda")
+    gp.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+    yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+    assert gp.get_error() == 0
+    gb, ob = dump_bytes(gp, ids), op.slot_bytes(ids)
+    offs, _ = O.head_offsets(bits, row_bits=rb)
+    for h, b in enumerate(bits):                       # one head block at a time
+        sl = slice(int(offs[h]), int(offs[h]) + (O.block_bytes(b) if b else O.rows_block_bytes(rb[h])))
+        res = PH.compare_slots(gb[:, sl], ob[:, sl], [b], row_bits=rb[h:h + 1])
+        assert res["max_code_diff"] <= 1 and res["r_ulp"] <= PH.R_ULP, (h, res)
+        if b:
+            assert PH.impact_scales_ok(res), (h, res)
+            assert res["flips_near"] <= max(1, PH.CODE_FLIP_RATE_IMPACT * res["elements"]), (h, res)
+        else:
+            assert res["c_ulp"] <= PH.C_ULP, (h, res)
+            assert res["flips"] <= max(1, PH.CODE_FLIP_RATE * res["elements"]), (h, res)
+    assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL
+    gp.close()
