@@ -98,3 +98,38 @@ def test_rowbits_pool_plumbing():
     Q1, r1, c1 = pool.state(0, 1)
     assert np.array_equal(Q1, Qe) and np.array_equal(r1, re) and np.array_equal(c1, ce)
     assert np.array_equal(y[0, 1], y_fp[0, 0])
+
+
+def test_mixed_pool_with_impact_scores_dispatches_each_fit():
+    """One pool with a per-key-row head next to uniform heads and row-impact scores set: a KDA
+    step through the pool equals, head by head, the unquantized step followed by the head's own
+    fit -- the clip-free per-row fit for the per-row head, the impact-weighted fit for the
+    uniform heads (the impact scores do not reach the per-row head)."""
+    rng = np.random.default_rng(41)
+    H = 3
+    bits = [6, 0, 8]
+    rbs = np.stack([np.full(128, 6), rng.choice([4, 6, 8], 128), np.full(128, 8)]).astype(np.int32)
+    omega = np.exp(rng.normal(0, 1, (H, 128))).astype(f32)
+    pool = O.OraclePool(2, bits, H, 1, row_bits=rbs, impact=omega)
+    S = (rng.standard_normal((1, H, 128, 128)) * 0.3).astype(f32)
+    pool.load_fp32([1], S)
+    q = rng.standard_normal((1, H, 128)).astype(f32)
+    k = rng.standard_normal((1, H, 128)).astype(f32)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((1, H, 128)).astype(f32)
+    a = rng.uniform(0.5, 1, (1, H, 128)).astype(f32)
+    b = rng.uniform(0, 1, (1, H)).astype(f32)
+    before = [pool.state(1, h) for h in range(H)]
+    y = pool.decode_step([1], q, k, v, a, b)
+    for h in range(H):
+        Sx = np.ascontiguousarray(O.dequantize(*before[h])[None, None])
+        sl = slice(h, h + 1)
+        y_fp = O.fp_decode_step(Sx, 1, 1, q[:, sl], k[:, sl], v[:, sl], a[:, sl], b[:, sl], round_fp32=True)
+        S32 = Sx[0, 0].astype(f32)
+        if bits[h] == 0:
+            Qe, re, ce, _ = O.rows_quantize(S32, rbs[h])
+        else:
+            Qe, re, ce, _ = O.quantize_impact(S32, bits[h], O.impact_normalize(omega[h]))
+        Q1, r1, c1 = pool.state(1, h)
+        assert np.array_equal(Q1, Qe) and np.array_equal(r1, re) and np.array_equal(c1, ce), h
+        assert np.array_equal(y[0, h], y_fp[0, 0]), h
