@@ -58,6 +58,8 @@ def parse():
                          "kda: the KDA layer (per-channel gates)")
     ap.add_argument("--batch", type=int, default=1024, choices=[64, 256, 1024],
                     help="requests of the stack sweep")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the device-timed sweep of the other workloads after the headline line's legs")
     return ap.parse_args()
 
 
@@ -287,7 +289,7 @@ def run_reference(args):
     print(json.dumps(line))
 
 
-def run_stack(args):
+def _time_stack(batch: int, steps: int, warmup: int, clocks_too: bool = False) -> dict:
     """36-layer stack sweep: a step runs layers 0..35 in order, each a decode step of its own
     pool (per-layer allocation).  Timed twice on the device: 36 plain launches per step, and
     the step captured once as a CUDA graph and replayed."""
@@ -296,8 +298,7 @@ def run_stack(args):
     from quantized_gated_delta_b200 import stepq
     from quantized_gated_delta_b200 import workloads as W
 
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    w = W.make_workload(5, batch=args.batch)
+    w = W.make_workload(5, batch=batch)
     L = w.layers
     pools, bits_all = [], []
     for layer in range(L):
@@ -318,15 +319,16 @@ def run_stack(args):
             x = xs[layer]
             pools[layer].decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y)
 
-    for i in range(max(3, args.warmup)):
+    for i in range(max(3, warmup)):
         step(i)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    sampler = ClockSampler(0)
-    sampler.start()
+    sampler = ClockSampler(0) if clocks_too else None
+    if sampler:
+        sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -343,43 +345,136 @@ def run_stack(args):
         g.replay()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     ms_graph = e0.elapsed_time(e1)
-    clocks = sampler.stop()
+    clocks = sampler.stop() if sampler else None
     for p_ in pools:
         if p_.get_error() != 0:
             raise RuntimeError("device flag set in the stack sweep")
-    units = w.B * w.H * L * args.steps
-    value = units / (ms_graph / 1e3)
+    units = w.B * w.H * L * steps
     # the same pool with FP32 states (d_k x d_v float32 per head, no scales): the pages'
     # reference point for the state-pool memory
     fp32_bytes = int(L * w.num_slots * w.H * w.dk * w.dv * 4)
+    pool_bytes = int(sum(p_.total_bytes for p_ in pools))
     alg = sum(algorithmic_bytes_per_step(w, b) for b in bits_all)          # one step, all layers
     peak, peak_kind = peaks()
-    achieved = alg * args.steps / (ms_graph / 1e3) / 1e9
-    line = {"metric": "quantized-state updates/s (req·head·layer-step), 36-layer stack", "value": value,
-            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_graph / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "%s: %d layers x H=%d, Hk=%d, B=%d, per-layer allocation (6.0 avg), bf16 inputs"
-                                   % (w.name, L, w.H, w.Hk, w.B),
-                       "pool_bytes": int(sum(p_.total_bytes for p_ in pools)),
-                       "fp32_pool_bytes": fp32_bytes,
-                       "fp32_over_packed": fp32_bytes / float(sum(p_.total_bytes for p_ in pools)),
-                       "l2": "no flush: each layer's pool is re-read after the other 35 (stack > 126 MB L2)"},
-            "us_per_layer_step_graph": ms_graph * 1e3 / (args.steps * L),
-            "us_per_layer_step_plain": ms_plain * 1e3 / (args.steps * L),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "peak_source": peak_kind, "traffic": None,
-                         "algorithmic_bytes_per_step": alg, "kernel": "decode_kernel (36 launches per step)"},
-            "gpu_launches": args.steps * L, "clocks": clocks}
-    print(json.dumps(line))
+    achieved = alg * steps / (ms_graph / 1e3) / 1e9
     del g
     for p_ in pools:
         p_.close()
+    return {"workload": w.name, "w": w, "B": w.B, "L": L, "steps": steps, "ms_graph": ms_graph,
+            "ms_plain": ms_plain, "us_per_layer_step": ms_graph * 1e3 / (steps * L),
+            "us_per_layer_step_plain": ms_plain * 1e3 / (steps * L), "updates_per_s": units / (ms_graph / 1e3),
+            "achieved_gbs": achieved, "frac": achieved / peak, "peak": peak, "peak_kind": peak_kind,
+            "alg": alg, "pool_bytes": pool_bytes, "fp32_pool_bytes": fp32_bytes, "clocks": clocks}
+
+
+def run_stack(args):
+    """The 36-layer stack sweep as its own bench line (--workload stack)."""
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    r = _time_stack(args.batch, args.steps, args.warmup, clocks_too=True)
+    w = r["w"]
+    line = {"metric": "quantized-state updates/s (req·head·layer-step), 36-layer stack", "value": r["updates_per_s"],
+            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": r["ms_graph"] / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "%s: %d layers x H=%d, Hk=%d, B=%d, per-layer allocation (6.0 avg), bf16 inputs"
+                                   % (w.name, r["L"], w.H, w.Hk, w.B),
+                       "pool_bytes": r["pool_bytes"],
+                       "fp32_pool_bytes": r["fp32_pool_bytes"],
+                       "fp32_over_packed": r["fp32_pool_bytes"] / float(r["pool_bytes"]),
+                       "l2": "no flush: each layer's pool is re-read after the other 35 (stack > 126 MB L2)"},
+            "us_per_layer_step_graph": r["us_per_layer_step"],
+            "us_per_layer_step_plain": r["us_per_layer_step_plain"],
+            "roofline": {"bound": "hbm", "achieved": r["achieved_gbs"], "peak": r["peak"], "unit": "GB/s",
+                         "frac": r["frac"], "peak_source": r["peak_kind"], "traffic": None,
+                         "algorithmic_bytes_per_step": r["alg"], "kernel": "decode_kernel (36 launches per step)"},
+            "gpu_launches": args.steps * r["L"], "clocks": r["clocks"]}
+    print(json.dumps(line))
+
+
+def _time_pool_workload(config: int, variant: str, fit: str, steps: int) -> dict:
+    """Device time of one single-pool workload: a 16-step CUDA graph of decode steps replayed
+    (inputs resident in HBM, cycling through 4 sets), after 4 warm-up steps."""
+    import torch
+
+    from quantized_gated_delta_b200 import stepq
+    from quantized_gated_delta_b200 import workloads as W
+
+    w = W.make_workload(config, variant)
+    row_bits = None
+    if w.row_half_life is not None:
+        rb = stepq.stepq_allocate_bits(np.ravel(w.row_half_life[0]), None, (4, 6, 8), w.avg_bits)
+        row_bits = np.asarray(rb, np.uint8).reshape(w.H, w.dk)
+        bits = np.zeros(w.H, dtype=np.uint8)
+    elif w.head_bits is not None:
+        bits = np.asarray(w.head_bits[0], np.uint8)
+    elif w.n_pivots:
+        bits = np.asarray(stepq.stepq_allocate_bits_pivots(w.half_life[0], None, (4, 6, 8), w.avg_bits,
+                                                           w.n_pivots), np.uint8)
+    else:
+        bits = np.asarray(stepq.stepq_allocate_bits(w.half_life[0], None, (4, 6, 8), w.avg_bits), np.uint8)
+    pool = stepq.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype, row_bits=row_bits)
+    if fit == "impact":
+        pool.set_impact(W.impact_scores(w))
+    slots = torch.from_numpy(w.slot_ids).cuda()
+    sets = [{k: torch.from_numpy(W.as_device_dtype(w, v).view(np.int16)).cuda()
+             for k, v in W.step_inputs(w, t).items()} for t in range(4)]
+    y = torch.empty((w.B, w.H, w.dv), device="cuda")
+    stream = torch.cuda.current_stream()
+    for t in range(4):
+        x = sets[t]
+        pool.decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y, stream)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for t in range(GRAPH_CHUNK):
+                x = sets[t % 4]
+                pool.decode_step(slots, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y, side)
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, steps // GRAPH_CHUNK)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if pool.get_error() != 0:
+        raise RuntimeError("device flag set in the %s sweep" % w.name)
+    us = e0.elapsed_time(e1) * 1e3 / (reps * GRAPH_CHUNK)
+    alg = algorithmic_bytes_per_step(w, bits, pool.slot_stride)
+    peak, _ = peaks()
+    del g
+    pool.close()
+    return {"workload": w.name + (" (impact-weighted fit)" if fit == "impact" else ""), "B": w.B, "H": w.H,
+            "Hk": w.Hk, "steps": reps * GRAPH_CHUNK, "us_per_step": us, "updates_per_s": w.B * w.H / (us / 1e6),
+            "achieved_gbs": alg / (us / 1e6) / 1e9, "frac": alg / (us / 1e6) / 1e9 / peak,
+            "algorithmic_bytes_per_step": alg}
+
+
+def workload_sweep() -> list:
+    """The other workloads of the build, device-timed after the headline measurement: the
+    hybrid GDN layer, the KDA layer (per-head and per-key-row widths), the high-concurrency
+    pool's uniform 4-bit, FP16-pivot and impact-fit variants, and the 36-layer stack at three
+    batch sizes (per layer-step, as one CUDA graph per step)."""
+    out = []
+    for config, variant, fit, steps in ((2, "mixed6", "clipfree", 1024), (3, "mixed6", "clipfree", 1024),
+                                        (3, "rowbits", "clipfree", 512), (4, "uniform4", "clipfree", 512),
+                                        (4, "mixed6p", "clipfree", 512), (4, "mixed6", "impact", 512)):
+        out.append(_time_pool_workload(config, variant, fit, steps))
+    for batch in (64, 256, 1024):
+        r = _time_stack(batch, 16, 3)
+        out.append({k: r[k] for k in ("workload", "B", "steps", "us_per_layer_step", "updates_per_s",
+                                      "achieved_gbs", "frac", "pool_bytes", "fp32_pool_bytes")})
+    return out
 
 
 def main():
@@ -545,6 +640,10 @@ def main():
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and row_bits is None:
         base = cpu_baseline(w, bits, args.cpu_seconds)
+    sweep = None
+    if world == 1 and not args.no_sweep and args.workload == "pool" and args.variant == "mixed6" \
+            and args.fit == "clipfree":
+        sweep = workload_sweep()
 
     if rank == 0:
         line = {
@@ -571,6 +670,7 @@ def main():
             "gpu_launches": args.steps * (2 if int(np.sum(bits == 16)) else 1),   # + pivot kernel
             "clocks": clocks,
             "cpu_baseline": base,
+            "workloads": sweep,
         }
         print(json.dumps(line))
     pool.close()
