@@ -696,6 +696,57 @@ def test_checkpoint_restore_continues_bit_identically(S):
     b.close()
 
 
+@pytest.mark.parametrize("variant,fit", [("mixed6", "clipfree"), ("mixed6p", "clipfree"), ("mixed6", "impact")])
+def test_graph_replay_matches_eager_steps(S, variant, fit):
+    """The launch configuration the benchmark times: config-4 decode steps (512 requests on a
+    1024-slot pool) captured as one CUDA graph on a side stream, programmatic dependent
+    launches between the steps, the FP16 pivot heads' kernel on the pool's forked stream
+    (mixed6p), and the impact-weighted fit.  Replays of the graph must give the eager launches'
+    y and packed states bit for bit (the kernels are deterministic), so the oracle parity of
+    the eager path carries over to the timed path."""
+    w = W.make_workload(4, variant)
+    bits = PH.head_bits(w)
+    ids = slots_t(w.slot_ids)
+    a = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    b = S.Pool(w.num_slots, bits, w.Hk, w.gate_mode, w.in_dtype)
+    if fit == "impact":
+        scores = _impact_scores(np.random.default_rng(91), w.H)
+        a.set_impact(scores)
+        b.set_impact(scores)
+    xs = [PH.to_device(w, W.step_inputs(w, t), torch) for t in range(12)]
+    nstep = 4
+    ya = torch.empty((nstep, w.B, w.H, w.dv), device="cuda")
+    yb = torch.empty_like(ya)
+
+    def steps(pool, y, first):
+        for t in range(nstep):
+            x = xs[first + t]
+            pool.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"], y[t])
+
+    # both pools leave the zero state through the same eager steps (deterministic: identical)
+    steps(a, ya, 0)
+    steps(b, yb, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(ya, yb)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            steps(a, ya, 4)
+    torch.cuda.current_stream().wait_stream(side)
+    for rep in range(2):
+        graph.replay()
+        steps(b, yb, 4)
+        torch.cuda.synchronize()
+        assert torch.equal(ya, yb), rep
+        assert np.array_equal(dump_bytes(a, w.slot_ids), dump_bytes(b, w.slot_ids)), rep
+    assert a.get_error() == 0 and b.get_error() == 0
+    del graph
+    a.close()
+    b.close()
+
+
 def test_debug_mode_rejects_duplicate_slot_ids(S):
     """With STEPQ_DEBUG_SLOTS a step with a repeated or out-of-range slot id is refused before
     any device work (the states stay as they were); distinct ids give the same step as
