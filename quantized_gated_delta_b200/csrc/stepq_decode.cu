@@ -655,7 +655,11 @@ struct ItemLoop {
             const float4 kqv = *reinterpret_cast<const float4 *>(sc.kqw);
             const float kq = (kqv.x + kqv.y) + (kqv.z + kqv.w);
             const int valid = sc.meta[st].valid;
-            if (has_next) ok &= mbar_wait_bounded(&sc.full[(i + 1) % kStages], uint32_t((i + 1) / kStages) & 1u);
+            // one thread waits for the next item's stage: its copies become visible to that
+            // thread, and the block barrier that follows (barrier 1 of this item, or the one
+            // of an empty item) orders every other thread's reads of the stage after the wait
+            if (has_next && tid == DK)
+                ok &= mbar_wait_bounded(&sc.full[(i + 1) % kStages], uint32_t((i + 1) / kStages) & 1u);
             bool alive;
             if (!valid) {
                 alive = !__syncthreads_or(!ok);
