@@ -103,6 +103,42 @@ def recorded_traffic(workload_name: str):
     return None
 
 
+def copy_link_rates(hin, hout, reps: int = 20) -> dict:
+    """Copy rates between the device and the given pinned host buffers (the host-buffer leg's
+    own input image and y, since the rate depends on where the host pages sit): each direction
+    alone, then both at once on two streams, as in the leg."""
+    import torch
+    hin, hout = hin.view(torch.uint8).reshape(-1), hout.view(torch.uint8).reshape(-1)
+    h2d_bytes, d2h_bytes = hin.numel(), hout.numel()
+    din = torch.empty(h2d_bytes, dtype=torch.uint8, device="cuda")
+    dout = torch.empty(d2h_bytes, dtype=torch.uint8, device="cuda")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def timed(do_in, do_out):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for _ in range(reps):
+            if do_in:
+                with torch.cuda.stream(s_in):
+                    din.copy_(hin, non_blocking=True)
+            if do_out:
+                with torch.cuda.stream(s_out):
+                    hout.copy_(dout, non_blocking=True)
+        torch.cuda.current_stream().wait_stream(s_in)
+        torch.cuda.current_stream().wait_stream(s_out)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3 / reps
+
+    timed(True, True)                                # warm-up
+    t_in, t_out, t_both = timed(True, False), timed(False, True), timed(True, True)
+    return {"h2d_gbs": h2d_bytes / t_in / 1e9, "d2h_gbs": d2h_bytes / t_out / 1e9,
+            "both_h2d_gbs": h2d_bytes / t_both / 1e9, "both_d2h_gbs": d2h_bytes / t_both / 1e9}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
@@ -603,9 +639,10 @@ def main():
     # (stepq_host_image_layout), so the call copies them in one transfer
     offs, img_bytes = pool.host_image_layout(w.B)
     names = ("slots", "q", "k", "v", "alpha", "beta")
-    host = []
+    host, images = [], []
     for x in host_sets[:E2E_HOST_SETS]:
         img = torch.zeros(img_bytes, dtype=torch.uint8).pin_memory()
+        images.append(img)
         arrays = [np.ascontiguousarray(w.slot_ids, dtype=np.int32)] + \
                  [W.as_device_dtype(w, x[k]).view(np.int16) for k in names[1:]]
         views = {}
@@ -636,6 +673,10 @@ def main():
     torch.cuda.synchronize()
     ms_e2e = D.max_over_ranks(e0.elapsed_time(e1), "cuda")
     e2e_value = units_per_step * args.e2e_steps * world / (ms_e2e / 1e3)
+    link = copy_link_rates(images[0], y_host)
+    # what the leg can reach: the slowest of the kernel, the input copy and the y copy, the two
+    # copies running at once in opposite directions
+    bound_us = max(avg_kernel_s * 1e6, h2d / (link["both_h2d_gbs"] * 1e3), d2h / (link["both_d2h_gbs"] * 1e3))
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and row_bits is None:
@@ -660,6 +701,9 @@ def main():
                          "kernel": "decode_kernel", "avg_kernel_us": avg_kernel_s * 1e6},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps,
+                    "us_per_step": ms_e2e * 1e3 / args.e2e_steps,
+                    "copy_link": link, "bound_us_per_step": bound_us,
+                    "frac_of_bound": bound_us / (ms_e2e * 1e3 / args.e2e_steps),
                     "api": "stepq_decode_step_host: one pinned input image per step (stepq_host_image_layout), "
                            "one host-to-device and one device-to-host copy per step, copies of consecutive steps "
                            "overlapped"},
