@@ -341,6 +341,7 @@ int stepq_pool_head_offset(const stepq_pool *pool, int32_t h, size_t *offset)
 int stepq_pool_load_fp32(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const float *S,
                          stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_pool_load_fp32");
     int st = check_slots(pool, slot_ids, n);
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
@@ -353,6 +354,7 @@ int stepq_pool_load_fp32(stepq_pool *pool, const int32_t *slot_ids, int32_t n, c
 int stepq_pool_load_packed(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const uint8_t *bytes,
                            stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_pool_load_packed");
     int st = check_slots(pool, slot_ids, n);
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
@@ -365,6 +367,7 @@ int stepq_pool_load_packed(stepq_pool *pool, const int32_t *slot_ids, int32_t n,
 int stepq_pool_dump_fp32(const stepq_pool *pool, const int32_t *slot_ids, int32_t n, float *S_out,
                          stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_pool_dump_fp32");
     int st = check_slots(pool, slot_ids, n);
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
@@ -377,6 +380,7 @@ int stepq_pool_dump_fp32(const stepq_pool *pool, const int32_t *slot_ids, int32_
 int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot_ids, int32_t n, uint8_t *bytes_out,
                            stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_pool_dump_packed");
     int st = check_slots(pool, slot_ids, n);
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
@@ -389,6 +393,7 @@ int stepq_pool_dump_packed(const stepq_pool *pool, const int32_t *slot_ids, int3
 int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q, const void *k,
                       const void *v, const void *alpha, const void *beta, float *y, stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_decode_step");
     int st = check_slots(pool, slot_ids, n);
     if (st != STEPQ_OK) return st;
     if (n == 0) return STEPQ_OK;
@@ -406,6 +411,7 @@ int stepq_decode_step(stepq_pool *pool, const int32_t *slot_ids, int32_t n, cons
 int stepq_decode_step_host(stepq_pool *pool, const int32_t *slot_ids, int32_t n, const void *q, const void *k,
                            const void *v, const void *alpha, const void *beta, float *y, stepq_stream stream)
 {
+    const stepq::NvtxRange range("stepq_decode_step_host");
     if (!pool || n < 0 || n > pool->num_slots || n > 65535) return STEPQ_INVALID_ARG;
     int st = check_device(pool);
     if (st != STEPQ_OK) return st;

@@ -1164,6 +1164,7 @@ extern "C" int stepq_decode_step_noalloc(const stepq_pool_desc *desc, uint8_t *s
                                          const void *beta, float *y, int32_t *flag_out, stepq_stream stream)
 {
     using namespace stepq;
+    const NvtxRange range("stepq_decode_step_noalloc");
     if (!desc || !desc->head_bits || n < 0) return STEPQ_INVALID_ARG;
     if (desc->num_slots <= 0 || desc->num_heads <= 0 || desc->num_key_heads <= 0) return STEPQ_INVALID_ARG;
     if (desc->num_heads % desc->num_key_heads != 0) return STEPQ_INVALID_ARG;
