@@ -112,6 +112,8 @@ def flips_off_tie(gpu_bytes, ora_before, bits, Hk, x, dk=128, dv=128):
     ora_before [n, slot_stride], and the inputs x of those n requests, GDN) gives the
     updated state before rounding and the fitted r, c; a code may differ by one only where
     |S / (r c)| lies within TIE_DIST of a half-integer (both roundings are then correct).
+    x["alpha"][s, h] is a head's gate (GDN) or its 128 per-channel gates (KDA).  FP16 pivot
+    heads (width 16) hold no codes and are skipped; compare_slots checks them.
     Returns (count of differing codes off a tie, largest code difference)."""
     offs, _ = O.head_offsets(bits, dk, dv)
     H = len(bits)
@@ -119,6 +121,8 @@ def flips_off_tie(gpu_bytes, ora_before, bits, Hk, x, dk=128, dv=128):
     for s in range(gpu_bytes.shape[0]):
         for h, b in enumerate(bits):
             b = int(b)
+            if b == 16:
+                continue
             n = O.block_bytes(b, dk, dv)
             Q0, r0, c0 = O.split_block(ora_before[s, offs[h]:offs[h] + n], b, dk, dv)
             g = h // (H // Hk)

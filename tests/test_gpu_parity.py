@@ -348,6 +348,53 @@ def test_key_head_groups_vs_oracle(S, H, Hk, gate, n):
     assert PH.y_max_rel(yg, yo) <= PH.Y_MAX_REL
 
 
+@pytest.mark.parametrize("bits,Hk,gate,n,num_slots,dtype", [
+    ([6], 1, 0, 1, 1, 0),                 # one request, one head, a one-slot pool
+    ([8, 4], 1, 1, 1, 3, 1),              # one request, a key head shared by two heads, KDA, bf16
+    ([8] * 6, 3, 0, 3, 7, 1),             # every head 8-bit
+    ([4] * 5 + [16], 1, 1, 2, 2, 0),      # every quantized head 4-bit plus a pivot, full pool
+], ids=["n1-h1-slots1", "n1-h2-kda-bf16", "all8bit", "all4bit-pivot-fullpool"])
+def test_smallest_shapes_vs_oracle(S, bits, Hk, gate, n, num_slots, dtype):
+    """The degenerate end of the shape range: one request, one head, a pool with a single
+    slot, a pool whose slots are all active, and pools of a single width.  Far fewer items
+    than resident CTAs, so most CTAs of the persistent grid have nothing to do.  Two steps
+    against the oracle.  Codes are checked element by element: each equals the oracle's or
+    differs by one where the oracle's S / (r c) is at a rounding tie.  A flip-rate bar does
+    not fit a pool of 8-bit heads only: the window of near-ties grows with qmax, and fp32
+    arithmetic against the fp64 oracle flips about 1.4e-5 of such codes, all at ties."""
+    rng = np.random.default_rng(7 * n + len(bits) + 3 * gate)
+    H = len(bits)
+    ids = rng.permutation(num_slots)[:n].astype(np.int32)
+    op = O.OraclePool(num_slots, bits, Hk, gate)
+    op.load_fp32(ids, random_states(rng, n, H, steps=5))
+    gp = S.Pool(num_slots, bits, Hk, gate, dtype)
+    load_bytes(gp, ids, op.slot_bytes(ids))
+    for step in range(2):
+        x = dict(q=_unit_rows(rng, (n, Hk)), k=_unit_rows(rng, (n, Hk)),
+                 v=rng.standard_normal((n, H, 128)).astype(f32),
+                 alpha=rng.uniform(0.7, 1, (n, H) if gate == 0 else (n, H, 128)).astype(f32),
+                 beta=rng.uniform(0.1, 0.9, (n, H)).astype(f32))
+        if dtype == S.STEPQ_DTYPE_BF16:         # both sides take the bf16-rounded inputs
+            x = {k_: W.round_bf16(v_) for k_, v_ in x.items()}
+            tx = {k_: dev(W.to_bf16_bits(v_).view(np.int16)) for k_, v_ in x.items()}
+        else:
+            tx = {k_: dev(v_) for k_, v_ in x.items()}
+        y = torch.empty((n, H, 128), device="cuda")
+        gp.decode_step(slots_t(ids), tx["q"], tx["k"], tx["v"], tx["alpha"], tx["beta"], y)
+        before = op.slot_bytes(ids)
+        yo = op.decode_step(ids, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+        sg = dump_bytes(gp, ids)
+        res = PH.compare_slots(sg, op.slot_bytes(ids), bits)
+        assert PH.pivots_ok(res), (step, res["pivot_flips"], res["pivot_elements"], res["pivot_ulp"])
+        off_tie, worst = PH.flips_off_tie(sg, before, bits, Hk, x)
+        assert worst <= 1 and off_tie == 0, (step, worst, off_tie, res["flips"])
+        assert res["r_ulp"] <= PH.R_ULP and res["c_ulp"] <= PH.C_ULP, step
+        assert PH.y_max_rel(y.cpu().numpy(), yo) <= PH.Y_MAX_REL, step
+        load_bytes(gp, ids, op.slot_bytes(ids))  # the next step starts from identical states
+    assert gp.get_error() == 0
+    gp.close()
+
+
 def test_kda_equal_gates_gqa_and_bf16_identities(S):
     """Bit identities on the GPU: KDA with equal per-channel gates = GDN; Hk = 2 with
     H = 4 = repeated key heads; bf16 inputs = the same values given as fp32."""
