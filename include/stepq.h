@@ -24,6 +24,9 @@
  *     debug mode of stepq_pool_set_debug rejects them).  An out-of-range slot id is skipped by
  *     the kernels and raises the pool's sticky device flag (read with stepq_pool_get_error);
  *     kernels never trap.
+ *   - Each data-path call (load, dump, decode) opens an NVTX range named after itself over its
+ *     argument checks and enqueue, so a profiler that records NVTX can attribute the call's
+ *     kernels to it; with no tool attached this costs a few nanoseconds.
  *
  * State and layout (shared by every call; the pages leave the format open)
  *   - value head h of request b lives in slot s = slot_ids[b]; key head g(h) = h / (H / H_k)
