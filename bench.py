@@ -497,7 +497,7 @@ def _time_pool_workload(config: int, variant: str, fit: str, steps: int) -> dict
 
 
 def workload_sweep() -> list:
-    """The other workloads of the build, device-timed after the headline measurement: the
+    """The other workloads, device-timed after the headline measurement: the
     hybrid GDN layer, the KDA layer (per-head and per-key-row widths), the high-concurrency
     pool's uniform 4-bit, FP16-pivot and impact-fit variants, and the 36-layer stack at three
     batch sizes (per layer-step, as one CUDA graph per step)."""

@@ -132,7 +132,7 @@ def _loguniform_half_life(seed: int, layers: int, H: int) -> np.ndarray:
 
 
 def make_workload(config: int, variant: str = "mixed6", batch: int | None = None) -> Workload:
-    """The five serving workloads (sizes as listed in the build's baseline).
+    """The five serving workloads, shaped like the pages' many-request hybrid-model serving.
 
     1  GDN toy: B=4, H=Hk=4, T=16, fp32, half-lives [2,32,512,4096], bits [4,6,8,8], seed 0
     2  GDN hybrid layer: B=64, H=32, Hk=16, T=64, bf16, log-uniform half-lives, 6-bit nominal

@@ -8,7 +8,7 @@ Two drivers are built here with the sanitizers on:
   creation and destruction, an allocation failure injected at each device allocation of
   pool creation (STEPQ_OUT_OF_MEMORY, no leak), the slot-id debug mode, the host-buffer
   staging path, the impact-score normalization and the allocator.
-A sanitizer report or a failed check makes the driver exit non-zero.
+A sanitizer report or a failed check makes the driver program exit non-zero.
 """
 import os
 import shutil
