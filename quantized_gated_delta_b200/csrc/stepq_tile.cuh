@@ -210,12 +210,23 @@ __device__ __forceinline__ void reduce_scatter(float (&a)[NV], int lane)
         const int o = OFF0 >> s;
         const int h = (NV >> s) / 2;
         const bool upper = (lane & o) != 0;
+        float keep[NV / 2], recv[NV / 2];
 #pragma unroll
         for (int i = 0; i < h; ++i) {
             const float send = upper ? a[i] : a[i + h];
-            const float keep = upper ? a[i + h] : a[i];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-            a[i] = MAX ? fmaxf(keep, recv) : keep + recv;
+            keep[i] = upper ? a[i + h] : a[i];
+            recv[i] = __shfl_xor_sync(0xffffffffu, send, o);
+        }
+#pragma unroll
+        for (int i = 0; i < h; i += 2) {
+            if (MAX || i + 1 >= h) {
+                a[i] = MAX ? fmaxf(keep[i], recv[i]) : keep[i] + recv[i];
+                if (i + 1 < h) a[i + 1] = fmaxf(keep[i + 1], recv[i + 1]);
+            } else {                        // two sums in one f32x2 add (the same IEEE adds)
+                const float2 t = fadd2(make_float2(keep[i], keep[i + 1]), make_float2(recv[i], recv[i + 1]));
+                a[i] = t.x;
+                a[i + 1] = t.y;
+            }
         }
     }
 }
